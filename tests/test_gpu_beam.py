@@ -1,0 +1,312 @@
+"""GPU parity of the trie builder, beam_step and beam_finalize against the oracle.
+
+Every call goes through the C ABI (ctypes binding). Inputs are seeded: the
+catalog comes from sidgen.host, logits from the device twin of the generator
+(bit-identical to the host twin the oracle uses).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from sidgen import host
+from sidgen.workloads import WORKLOADS
+
+from parity import TOL, compare_step, oracle_search_with_gaps, run_gpu_search, to_host_logits
+
+pytestmark = pytest.mark.gpu
+
+_catalog_cache = {}
+
+
+def _catalog(cfg):
+    if cfg not in _catalog_cache:
+        w = WORKLOADS[cfg]
+        cat = w.catalog()
+        _catalog_cache[cfg] = (cat, oracle.OracleTrie(cat, w.codes_per_level))
+    return _catalog_cache[cfg]
+
+
+@pytest.fixture(scope="module")
+def tcb():
+    import trie_constrained_beam_b200 as m
+    from trie_constrained_beam_b200 import build
+    from sidgen import device
+    build.build()
+    device.build()
+    return m
+
+
+def _host(t):
+    return t.cpu().numpy()
+
+
+# ---------------------------------------------------------------- trie
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_trie_matches_oracle(tcb, cfg):
+    import torch
+    w = WORKLOADS[cfg]
+    cat, otrie = _catalog(cfg)
+    # Duplicate some rows to exercise de-duplication and the first-row map.
+    dup = np.concatenate([cat, cat[::7]])
+    gtrie = tcb.sid_trie_build(dup, w.codes_per_level, w.layouts)
+    otrie2 = oracle.OracleTrie(dup, w.codes_per_level)
+    for lv in range(w.depth + 1):
+        n, lay, nb = tcb.sid_trie_info(gtrie, lv)
+        assert n == otrie2.n_nodes(lv)
+    N = otrie2.leaves.shape[0]
+    codes = torch.empty((N, w.depth), dtype=torch.int32, device="cuda")
+    rows = torch.empty((N,), dtype=torch.int32, device="cuda")
+    tcb.sid_trie_leaf_codes(gtrie, codes)
+    tcb.sid_trie_leaf_rows(gtrie, rows)
+    assert np.array_equal(_host(codes), otrie2.leaves)
+    assert np.array_equal(_host(rows), otrie2.leaf_rows)
+
+
+# ---------------------------------------------------------------- step-local parity
+def _step_local(tcb, cfg, R=None, n=None, layouts="cfg", dtype=None, ld_pad=0):
+    w = WORKLOADS[cfg]
+    cat, otrie = _catalog(cfg)
+    R = R or w.R
+    n = n or w.n
+    dtype = dtype or w.dtype
+    lays = w.layouts if layouts == "cfg" else layouts
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, lays)
+    checked = []
+
+    def on_step(t, logits, ps, pn, B_in, out):
+        g = {k: _host(v).reshape(R, n) for k, v in out.items()}
+        exact = compare_step(g, otrie, t, to_host_logits(logits, w.V), _host(ps), _host(pn),
+                             R, B_in, n, w.V)
+        checked.append(exact)
+
+    run_gpu_search(gtrie, R, n, w.depth, w.V, w.logits_seed, w.sigma, dtype, ld_pad=ld_pad,
+                   on_step=on_step)
+    assert len(checked) == w.depth
+    return checked
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_step_local_parity_full_size(tcb, cfg):
+    exact = _step_local(tcb, cfg)
+    assert sum(exact) > 0
+
+
+def test_step_local_parity_padded_ld_and_fp32_config3_shape(tcb):
+    _step_local(tcb, 3, R=8, n=64, dtype="f32", ld_pad=37)
+
+
+# ---------------------------------------------------------------- end to end
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_end_to_end_parity(tcb, cfg):
+    w = WORKLOADS[cfg]
+    cat, otrie = _catalog(cfg)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    _, sids, leaf, scores = run_gpu_search(gtrie, w.R, w.n, w.depth, w.V, w.logits_seed, w.sigma,
+                                           w.dtype)
+    ref = oracle_search_with_gaps(otrie, w.R, w.n, w.depth, w.V, w.logits_seed, w.sigma, w.dtype)
+    sids, leaf, scores = _host(sids), _host(leaf), _host(scores).astype(np.float64)
+    catalog = {tuple(s) for s in otrie.leaves.tolist()}
+    compared = 0
+    for r in range(w.R):
+        # Every GPU beam is a catalog SID (invalid rate 0) and its leaf id matches.
+        for k in range(w.n):
+            if leaf[r, k] >= 0:
+                assert tuple(sids[r, k]) in catalog
+                assert tuple(otrie.leaves[leaf[r, k]]) == tuple(sids[r, k])
+        np.testing.assert_allclose(scores[r], ref["score"][r], atol=TOL * w.depth, rtol=0)
+        if ref["min_gap"][r] > 10 * TOL * w.depth:
+            os_ = ref["score"][r]
+            for k in range(w.n):
+                lo = k == 0 or os_[k - 1] - os_[k] > TOL * w.depth
+                hi = k == w.n - 1 or os_[k] - os_[k + 1] > TOL * w.depth
+                if lo and hi:
+                    assert np.array_equal(sids[r, k], ref["sids"][r, k])
+                    assert leaf[r, k] == ref["leaf"][r, k]
+            compared += 1
+    assert compared >= w.R // 2
+
+
+def test_exhaustive_beam_equals_brute_force(tcb):
+    """Config-1 catalog with beam 2000 >= |catalog|: the search returns every SID,
+    scored by the exhaustive sum of full-codebook log-softmax terms."""
+    import torch
+    w = WORKLOADS[1]
+    cat, otrie = _catalog(1)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    n = 2000
+    _, sids, leaf, scores = run_gpu_search(gtrie, 1, n, w.depth, w.V, w.logits_seed, w.sigma,
+                                           w.dtype)
+    leaves = otrie.leaves
+    brute = np.zeros(leaves.shape[0])
+    for lv in range(w.depth):
+        z = host.row_logits(w.logits_seed, host.prefix_hashes(leaves[:, :lv]), w.V, w.sigma)
+        lp = torch.log_softmax(torch.from_numpy(z.astype(np.float64)), dim=1).numpy()
+        brute += lp[np.arange(leaves.shape[0]), leaves[:, lv]]
+    order = np.argsort(-brute, kind="stable")
+    got_leaf = _host(leaf)[0]
+    assert sorted(got_leaf.tolist()) == list(range(leaves.shape[0]))
+    np.testing.assert_allclose(_host(scores)[0], brute[order], atol=TOL * w.depth, rtol=0)
+    gaps = brute[order][:-1] - brute[order][1:]
+    for k in range(leaves.shape[0]):
+        lo = k == 0 or gaps[k - 1] > TOL * w.depth
+        hi = k == leaves.shape[0] - 1 or gaps[k] > TOL * w.depth
+        if lo and hi:
+            assert got_leaf[k] == order[k]
+
+
+# ---------------------------------------------------------------- layouts, modes, ties
+def test_layout_invariance_dense_vs_csr(tcb):
+    import torch
+    w = WORKLOADS[2]
+    cat, _ = _catalog(2)
+    res = []
+    for lay in ([1] * w.depth, [2] * w.depth, None):
+        gtrie = tcb.sid_trie_build(cat, w.codes_per_level, lay)
+        _, sids, leaf, scores = run_gpu_search(gtrie, 8, 32, w.depth, w.V, w.logits_seed,
+                                               w.sigma, w.dtype)
+        res.append((_host(sids), _host(leaf), _host(scores)))
+        torch.cuda.synchronize()
+    for other in res[1:]:
+        for a, b in zip(res[0], other):
+            assert np.array_equal(a, b)
+
+
+def test_unconstrained_mode_matches_oracle(tcb):
+    import torch
+    R, B_in, n, V = 5, 12, 40, 300
+    rng = np.random.default_rng(11)
+    z = rng.normal(0, 2, size=(R * B_in, V)).astype(np.float32)
+    ps = rng.normal(-4, 1, size=R * B_in).astype(np.float32)
+    ps[3] = -np.inf
+    ld = 304
+    zt = torch.zeros((R * B_in, ld), dtype=torch.float32, device="cuda")
+    zt[:, :V] = torch.from_numpy(z).cuda()
+    out = dict(score=torch.empty(R * n, device="cuda"),
+               parent=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               code=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               node=torch.empty(R * n, dtype=torch.int32, device="cuda"))
+    ws = torch.zeros(tcb.beam_step_workspace_size(R, B_in, n, V), dtype=torch.uint8, device="cuda")
+    tcb.beam_step(None, 0, zt, torch.from_numpy(ps).cuda(), None, R, B_in, n, V, out["score"],
+                  out["parent"], out["code"], out["node"], ws)
+    g = {k: _host(v).reshape(R, n) for k, v in out.items()}
+    compare_step(g, None, 0, z, ps, np.zeros(R * B_in, dtype=np.int64), R, B_in, n, V)
+
+
+def _one_step(tcb, trie, step, z, ps, pn, R, B_in, n, V, dtype="f32"):
+    import torch
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    zt = torch.from_numpy(z).cuda().to(tdt)
+    out = dict(score=torch.empty(R * n, device="cuda"),
+               parent=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               code=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               node=torch.empty(R * n, dtype=torch.int32, device="cuda"))
+    ws = torch.zeros(tcb.beam_step_workspace_size(R, B_in, n, V), dtype=torch.uint8, device="cuda")
+    tcb.beam_step(trie, step, zt, torch.from_numpy(np.asarray(ps, np.float32)).cuda(),
+                  torch.from_numpy(np.asarray(pn, np.int32)).cuda(), R, B_in, n, V,
+                  out["score"], out["parent"], out["code"], out["node"], ws)
+    return {k: _host(v).reshape(R, n) for k, v in out.items()}, ws
+
+
+def test_all_equal_logits_pick_lexicographic_first(tcb):
+    sids = np.array([[2, 3], [0, 1], [3, 1], [1, 0], [0, 3], [2, 2]])
+    gtrie = tcb.sid_trie_build(sids, [4, 4], [2, 2])
+    g, _ = _one_step(tcb, gtrie, 1, np.zeros((3, 4), np.float32), np.full(3, -np.log(4)),
+                     [0, 1, 2], 1, 3, 3, 4)
+    assert g["parent"][0].tolist() == [0, 0, 1]
+    assert g["code"][0].tolist() == [1, 3, 0]
+    assert g["node"][0].tolist() == [0, 1, 2]
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_quantised_logits_many_ties_bit_exact(tcb, layout):
+    """Identical rows with logits on a coarse grid: candidates tie exactly inside
+    and across rows, and the (parent, code) tie-break decides everything."""
+    rng = np.random.default_rng(5)
+    Vs = [64, 64]
+    cat = host.draw_catalog(77, 1500, Vs)
+    otrie = oracle.OracleTrie(cat, Vs)
+    gtrie = tcb.sid_trie_build(cat, Vs, [layout, layout])
+    R, B_in, n, V = 3, 20, 150, 64
+    row = rng.integers(-2, 3, size=V).astype(np.float32) * 0.5
+    z = np.tile(row, (R * B_in, 1))
+    ps = np.zeros(R * B_in, np.float32)
+    pn = rng.integers(0, otrie.n_nodes(1), size=R * B_in)
+    g, _ = _one_step(tcb, gtrie, 1, z, ps, pn, R, B_in, n, V)
+    ref = oracle.beam_step(otrie, 1, z, ps, pn, R, B_in, n, V)
+    for key in ("parent", "code", "node"):
+        assert np.array_equal(g[key], ref[key])
+    np.testing.assert_allclose(g["score"], ref["score"], atol=TOL)
+
+
+# ---------------------------------------------------------------- randomised sweep
+@pytest.mark.parametrize("seed", range(40))
+def test_random_sweep(tcb, seed):
+    rng = np.random.default_rng(9000 + seed)
+    depth = int(rng.integers(1, 5))
+    V = int(rng.choice([1, 2, 5, 8, 31, 33, 64, 100, 256, 1000, 2049]))
+    space = V ** depth
+    n_cat = int(min(space, rng.integers(1, 3000)))
+    cat = host.draw_catalog(seed, n_cat, [V] * depth)
+    otrie = oracle.OracleTrie(cat, [V] * depth)
+    lay = [int(rng.choice([0, 1, 2])) for _ in range(depth)]
+    gtrie = tcb.sid_trie_build(cat, [V] * depth, lay)
+    R = int(rng.integers(1, 9))
+    n = int(rng.choice([1, 2, 7, 32, 100, 513]))
+    dtype = "bf16" if rng.random() < 0.5 else "f32"
+    checked = []
+
+    def on_step(t, logits, ps, pn, B_in, out):
+        g = {k: _host(v).reshape(R, n) for k, v in out.items()}
+        compare_step(g, otrie, t, to_host_logits(logits, V), _host(ps), _host(pn), R, B_in, n, V)
+        checked.append(t)
+
+    run_gpu_search(gtrie, R, n, depth, V, 500 + seed, float(rng.uniform(0.5, 4.0)), dtype,
+                   ld_pad=int(rng.integers(0, 9)), on_step=on_step)
+    assert len(checked) == depth
+
+
+# ---------------------------------------------------------------- determinism, errors
+def test_repeated_runs_bitwise_equal(tcb):
+    w = WORKLOADS[2]
+    cat, _ = _catalog(2)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    first = None
+    for _ in range(10):
+        _, sids, leaf, scores = run_gpu_search(gtrie, w.R, w.n, w.depth, w.V, w.logits_seed,
+                                               w.sigma, w.dtype)
+        cur = (_host(sids), _host(leaf), _host(scores))
+        if first is None:
+            first = cur
+        for a, b in zip(first, cur):
+            assert np.array_equal(a, b)
+
+
+def test_error_conventions(tcb):
+    import torch
+    sids = np.array([[0, 1], [1, 0]])
+    gtrie = tcb.sid_trie_build(sids, [2, 2])
+    z = torch.zeros((2, 4), device="cuda")
+    ps = torch.zeros(2, device="cuda")
+    pn = torch.zeros(2, dtype=torch.int32, device="cuda")
+    o = [torch.empty(2, device="cuda")] + [torch.empty(2, dtype=torch.int32, device="cuda")
+                                           for _ in range(3)]
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tcb.SidbeamError) as e:
+        tcb.beam_step(gtrie, 1, z, ps, pn, 1, 2, 2, 2, *o, small)
+    assert e.value.status == -4
+    ws = torch.zeros(tcb.beam_step_workspace_size(1, 2, 2, 2), dtype=torch.uint8, device="cuda")
+    with pytest.raises(tcb.SidbeamError) as e:           # V disagrees with the trie
+        tcb.beam_step(gtrie, 1, z, ps, pn, 1, 2, 2, 3, *o, ws)
+    assert e.value.status == -1
+    with pytest.raises(tcb.SidbeamError) as e:           # misaligned leading dimension
+        tcb.beam_step(gtrie, 1, z, ps, pn, 1, 2, 2, 2, *o, ws, ld=3)
+    assert e.value.status == -3
+    with pytest.raises(tcb.SidbeamError) as e:           # code outside [0, V)
+        tcb.sid_trie_build(np.array([[0, 2]]), [2, 2])
+    assert e.value.status == -2
+    # A node id past the level's node count: the row is skipped and the status reports it.
+    bad = torch.tensor([0, 7], dtype=torch.int32, device="cuda")
+    tcb.beam_step(gtrie, 1, z, ps, bad, 1, 2, 2, 2, *o, ws)
+    assert tcb.sidbeam_get_device_status(ws) == -7
+    assert tcb.sidbeam_get_device_status(ws) == 0
+    assert _host(o[1]).tolist()[0] == 0    # row 0 (node (0,)) still expanded

@@ -1,0 +1,226 @@
+// catalog_score_topk: one-pass scoring of every catalog SID, then top-K.
+//
+// SPRINT (paper summary), inference paragraph: every valid SID of the prefix
+// trie is scored by the sum of its tokens' per-position log-probabilities (a
+// lookup in an L-by-M table per request), and the K best are returned.
+//
+// (request, leaf) pairs are laid out request-major and split evenly over the
+// CTAs, exactly like beam rows in beam_step. A CTA keeps the current
+// request's table in shared memory, each warp scores 32 leaves at a time from
+// the SoA leaf codes (coalesced uint16 loads), and candidates go through the
+// same warp / CTA / request top-n machinery as beam_step (topn.cuh).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "device_utils.cuh"
+#include "internal.h"
+#include "launch.h"
+#include "topn.cuh"
+
+namespace sidbeam {
+namespace {
+
+using namespace dev;
+
+constexpr int kScoreWarps = 8;
+
+struct ScoreConfig {
+  int W, Cw, ctas_per_sm;
+  int off_ctl, off_chist, off_whist, off_table, off_wkeys, off_wvals, smem_bytes;
+};
+
+struct ScoreArgs {
+  const uint16_t* leaf_codes;  // [depth][stride]
+  int64_t stride;
+  int64_t N;
+  int depth;
+  const float* logp;  // [R][depth][Vmax]
+  int Vmax;
+  int K;
+  float* out_scores;
+  int32_t* out_leaf;
+  uint32_t* status;
+  uint32_t* tickets;
+  unsigned long long* request_thr;
+  uint32_t* part_count;
+  unsigned long long* part_keys;
+  int32_t* part_vals;
+  Partition part;
+  ScoreConfig cfg;
+};
+
+struct ScoreWriter {
+  float* scores;
+  int32_t* leaf;
+  int K;
+  __device__ __forceinline__ void operator()(int r, int i, uint64_t key, int32_t, bool valid) const {
+    const size_t o = static_cast<size_t>(r) * K + i;
+    scores[o] = valid ? key_score(key) : __int_as_float(0xFF800000);
+    leaf[o] = valid ? static_cast<int32_t>(key_idx(key)) : -1;
+  }
+};
+
+__global__ void __launch_bounds__(kScoreWarps * 32)
+    catalog_score_kernel(const __grid_constant__ ScoreArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const ScoreConfig& cfg = a.cfg;
+  SelCtl* ctl = reinterpret_cast<SelCtl*>(smem + cfg.off_ctl);
+  uint32_t* cta_hist = reinterpret_cast<uint32_t*>(smem + cfg.off_chist);
+  uint32_t* whist = reinterpret_cast<uint32_t*>(smem + cfg.off_whist);
+  float* table = reinterpret_cast<float*>(smem + cfg.off_table);
+  uint64_t* wkeys = reinterpret_cast<uint64_t*>(smem + cfg.off_wkeys);
+  int32_t* wvals = reinterpret_cast<int32_t*>(smem + cfg.off_wvals);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Team team{static_cast<int>(threadIdx.x), cfg.W * 32, warp, lane, cfg.W};
+  if (threadIdx.x == 0) {
+    ctl->cta_thr = 0ull;
+    ctl->abort_flag = 0;
+    ctl->counter = 0;
+  }
+  WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw, wvals + static_cast<size_t>(warp) * cfg.Cw,
+             whist + warp * 256, cfg.Cw, 0, 0ull};
+  const ScoreWriter writer{a.out_scores, a.out_leaf, a.K};
+  const int64_t row_lo = static_cast<int64_t>(blockIdx.x) * a.part.rows_per_cta;
+  const int64_t row_hi = min(a.part.total_rows, row_lo + a.part.rows_per_cta);
+  const int tsize = a.depth * a.Vmax;
+
+  for (int64_t seg_lo = row_lo; seg_lo < row_hi;) {
+    const int r = static_cast<int>(seg_lo / a.N);
+    const int64_t seg_hi = min(row_hi, static_cast<int64_t>(r + 1) * a.N);
+    const float* src = a.logp + static_cast<size_t>(r) * tsize;
+    for (int i = threadIdx.x; i < tsize; i += blockDim.x) table[i] = src[i];
+    team_sync(team);
+    const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
+    const int64_t j_lo = seg_lo - static_cast<int64_t>(r) * a.N;
+    const int64_t j_hi = seg_hi - static_cast<int64_t>(r) * a.N;
+    for (int64_t j0 = j_lo + static_cast<int64_t>(warp) * 32; j0 < j_hi;
+         j0 += static_cast<int64_t>(cfg.W) * 32) {
+      const int64_t j = j0 + lane;
+      const bool valid = j < j_hi;
+      float score = 0.f;
+      if (valid) {
+        score = table[a.leaf_codes[j]];
+        for (int l = 1; l < a.depth; ++l)
+          score += table[l * a.Vmax + a.leaf_codes[static_cast<int64_t>(l) * a.stride + j]];
+      }
+      const unsigned long long cthr =
+          *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+      if (cthr > wb.thr) wb.thr = cthr;
+      warp_offer(wb, valid, make_key(score, static_cast<uint32_t>(j)), static_cast<int32_t>(j),
+                 static_cast<uint32_t>(a.K), lane, sinks);
+    }
+    FlushArgs f;
+    f.n = a.K;
+    f.r = r;
+    f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(r);
+    f.G = a.part.contributors(r);
+    f.maxG = a.part.maxG;
+    f.part_keys = a.part_keys;
+    f.part_vals = a.part_vals;
+    f.part_count = a.part_count;
+    f.tickets = a.tickets;
+    f.request_thr = a.request_thr;
+    f.wkeys = wkeys;
+    f.cw = cfg.Cw;
+    f.sort_keys = wkeys;
+    f.sort_vals = wvals;
+    if (segment_flush(team, wb, ctl, cta_hist, f, writer)) return;
+    seg_lo = seg_hi;
+  }
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+bool choose_score_config(int depth, int Vmax, int K, ScoreConfig* out) {
+  ScoreConfig c{};
+  c.W = kScoreWarps;
+  int npow2 = 1;
+  while (npow2 < K) npow2 <<= 1;
+  c.Cw = std::max(round_up(K, 32) + 512, round_up((npow2 + c.W - 1) / c.W, 32));
+  int o = 0;
+  c.off_ctl = o;
+  o += round_up(static_cast<int>(sizeof(SelCtl)), 128);
+  c.off_chist = o;
+  o += 1024;
+  c.off_whist = o;
+  o += c.W * 1024;
+  c.off_table = o;
+  o = round_up(o + depth * Vmax * 4, 128);
+  c.off_wkeys = o;
+  o += c.W * c.Cw * 8;
+  c.off_wvals = o;
+  o += c.W * c.Cw * 4;
+  c.smem_bytes = round_up(o, 128);
+  if (c.smem_bytes > kSmemBudget) return false;
+  c.ctas_per_sm = std::max(1, std::min(4, kSmemBudget / c.smem_bytes));
+  *out = c;
+  return true;
+}
+
+}  // namespace
+}  // namespace sidbeam
+
+using namespace sidbeam;
+
+static int score_vmax(const sidbeam_trie* t) {
+  int v = 1;
+  for (int l = 0; l < t->depth; ++l) v = std::max(v, t->V[l]);
+  return v;
+}
+
+extern "C" size_t catalog_score_workspace_size(const sidbeam_trie* trie, int R, int K) {
+  if (!trie || R < 1 || K < 1 || K > SIDBEAM_MAX_BEAM) return 0;
+  ScoreConfig cfg;
+  if (!choose_score_config(trie->depth, score_vmax(trie), K, &cfg)) return 0;
+  const Partition p = make_partition(R, trie->n_leaves, device_sm_count() * cfg.ctas_per_sm);
+  return workspace_layout(R, p.maxG, K).total;
+}
+
+extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K,
+                                  float* out_scores, int32_t* out_leaf, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!trie || !logp || !out_scores || !out_leaf)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: NULL pointer argument");
+  if (R < 1 || K < 1 || K > SIDBEAM_MAX_BEAM)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: R=%d K=%d", R, K);
+  if (static_cast<int64_t>(R) * trie->n_leaves > (1ll << 40))
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: R * leaves too large");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return set_error(SIDBEAM_ERR_WORKSPACE, "catalog_score_topk: workspace must be 256-byte aligned");
+  ScoreArgs a{};
+  a.Vmax = score_vmax(trie);
+  if (!choose_score_config(trie->depth, a.Vmax, K, &a.cfg))
+    return set_error(SIDBEAM_ERR_INVALID_ARG,
+                     "catalog_score_topk: the [depth x V] table does not fit in shared memory");
+  a.leaf_codes = trie->leaf_codes;
+  a.stride = trie->leaf_codes_stride;
+  a.N = trie->n_leaves;
+  a.depth = trie->depth;
+  a.logp = logp;
+  a.K = K;
+  a.out_scores = out_scores;
+  a.out_leaf = out_leaf;
+  a.part = make_partition(R, trie->n_leaves, device_sm_count() * a.cfg.ctas_per_sm);
+  const WorkspaceLayout ws = workspace_layout(R, a.part.maxG, K);
+  if (!workspace || workspace_bytes < ws.total)
+    return set_error(SIDBEAM_ERR_WORKSPACE, "catalog_score_topk: workspace of %zu bytes, need %zu",
+                     workspace_bytes, ws.total);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<uint32_t*>(w + ws.status);
+  a.tickets = reinterpret_cast<uint32_t*>(w + ws.tickets);
+  a.request_thr = reinterpret_cast<unsigned long long*>(w + ws.request_thr);
+  a.part_count = reinterpret_cast<uint32_t*>(w + ws.part_count);
+  a.part_keys = reinterpret_cast<unsigned long long*>(w + ws.part_keys);
+  a.part_vals = reinterpret_cast<int32_t*>(w + ws.part_vals);
+  cudaError_t e = cudaFuncSetAttribute(catalog_score_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       a.cfg.smem_bytes);
+  if (e != cudaSuccess) return cuda_error(e, "catalog_score_topk: cudaFuncSetAttribute");
+  catalog_score_kernel<<<a.part.grid, a.cfg.W * 32, a.cfg.smem_bytes,
+                         static_cast<cudaStream_t>(stream)>>>(a);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SIDBEAM_OK : cuda_error(e, "catalog_score_topk: launch");
+}

@@ -1,0 +1,53 @@
+// Host-side internals of libsidbeam: the trie object and error reporting.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <string>
+
+#include "../../include/sidbeam.h"
+
+namespace sidbeam {
+
+// One expansion structure: level-t nodes (parents) -> level-(t+1) codes.
+struct StepTrie {
+  int layout = 0;               // SIDBEAM_LAYOUT_DENSE or SIDBEAM_LAYOUT_CSR
+  int V = 0;                    // codes at level t+1
+  int64_t n_parent = 0;         // P_t
+  int64_t n_child = 0;          // P_{t+1}
+  uint32_t* off = nullptr;      // [P_t + 1]: children of p are ids off[p] .. off[p+1]-1
+  uint32_t* mask = nullptr;     // dense: [P_t][mask_stride] bit c of row p = child code c
+  int mask_words = 0;           // ceil(V / 32)
+  int mask_stride = 0;          // mask_words rounded up to a multiple of 4 (16-byte rows)
+  uint16_t* codes = nullptr;    // CSR: [P_{t+1} + 8]: code of child id q (padded for 16-B loads)
+  size_t bytes = 0;
+};
+
+}  // namespace sidbeam
+
+struct sidbeam_trie {
+  int depth = 0;
+  int device = 0;
+  int V[SIDBEAM_MAX_DEPTH] = {};
+  int64_t n_nodes[SIDBEAM_MAX_DEPTH + 1] = {};
+  sidbeam::StepTrie steps[SIDBEAM_MAX_DEPTH];
+  int64_t n_leaves = 0;
+  int32_t* leaf_rows = nullptr;    // [n_leaves]
+  uint16_t* leaf_codes = nullptr;  // [depth][n_leaves + 8], SoA
+  int64_t leaf_codes_stride = 0;   // n_leaves + 8
+  size_t leaf_bytes = 0;
+};
+
+namespace sidbeam {
+
+int set_error(int status, const char* fmt, ...);
+int cuda_error(cudaError_t e, const char* what);
+int device_sm_count();
+
+// Device status word bits (first 4 bytes of a workspace).
+constexpr uint32_t kStatusBadNode = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+}  // namespace sidbeam

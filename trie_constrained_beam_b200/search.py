@@ -1,0 +1,59 @@
+"""Device buffers and the step loop of one constrained beam search.
+
+Orchestration only: every step is one ``beam_step`` call, the end is one
+``beam_finalize`` call. Step t reads the previous step's outputs as its parent
+rows (B_in = 1 at step 0: the root of every request, score 0), and writes its
+back-pointers straight into slice t of the [depth][R][n] history.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native
+
+
+class BeamSearch:
+    def __init__(self, trie, R: int, n: int, V, depth: int = None, device="cuda"):
+        self.trie = trie
+        self.depth = depth if depth is not None else trie.depth
+        self.V = list(V) if isinstance(V, (list, tuple)) else [int(V)] * self.depth
+        self.R, self.n = R, n
+        dev = torch.device(device)
+        self.root_scores = torch.zeros(R, dtype=torch.float32, device=dev)
+        self.root_nodes = torch.zeros(R, dtype=torch.int32, device=dev)
+        self.scores = torch.empty((self.depth, R * n), dtype=torch.float32, device=dev)
+        self.nodes = torch.empty((self.depth, R * n), dtype=torch.int32, device=dev)
+        self.bp_parent = torch.empty((self.depth, R, n), dtype=torch.int32, device=dev)
+        self.bp_code = torch.empty((self.depth, R, n), dtype=torch.int32, device=dev)
+        ws = 0
+        for t in range(self.depth):
+            ws = max(ws, native.beam_step_workspace_size(R, 1 if t == 0 else n, n, self.V[t]))
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=dev)
+        self.sids = torch.empty((R, n, self.depth), dtype=torch.int32, device=dev)
+        self.leaf = torch.empty((R, n), dtype=torch.int32, device=dev)
+
+    def rows(self, t: int) -> int:
+        return self.R * (1 if t == 0 else self.n)
+
+    def parents(self, t: int):
+        """(parent_scores, parent_nodes, B_in) of step t."""
+        if t == 0:
+            return self.root_scores, self.root_nodes, 1
+        return self.scores[t - 1], self.nodes[t - 1], self.n
+
+    def step(self, t: int, logits, stream=None):
+        ps, pn, B_in = self.parents(t)
+        native.beam_step(self.trie, t, logits, ps, pn, self.R, B_in, self.n, self.V[t],
+                         self.scores[t], self.bp_parent[t], self.bp_code[t], self.nodes[t],
+                         self.workspace, stream=stream)
+
+    def finalize(self, stream=None):
+        native.beam_finalize(self.depth, self.R, self.n, self.bp_parent, self.bp_code,
+                             self.nodes[self.depth - 1], self.sids, self.leaf, stream=stream)
+        return self.sids, self.leaf, self.scores[self.depth - 1].view(self.R, self.n)
+
+    def run(self, logits_for_step, stream=None):
+        """logits_for_step(t, search) -> logits tensor [rows(t), ld] for step t."""
+        for t in range(self.depth):
+            self.step(t, logits_for_step(t, self), stream=stream)
+        return self.finalize(stream=stream)
