@@ -1,0 +1,446 @@
+"""Benchmark: catalog-constrained wide-beam expansion on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One timed step = one whole constrained beam search of the wide-beam workload
+(16 requests x beam 512, depth 5, 4,096 codes per level, 8M-SID catalog with a
+dense trie on levels 1-2 and CSR below, bf16 logits): five beam_step launches
+plus beam_finalize. The per-step logits are the ones the search consumes (made
+once by the seeded generator, keyed by prefix hash) and are resident in HBM
+when the timed region starts; three rotating copies (3 x 256 MiB + step 0)
+keep every step's reads out of L2.
+
+Printed: one JSON line (rank 0). `value` = logits scored per second over all
+ranks (live rows x V summed over the five steps, per search). Multi-GPU runs
+are weak-scaled replicas: requests are independent, every rank searches its
+own batch, nothing crosses GPUs in the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "beam-step logits scored/sec & achieved HBM GB/s (% of B200 peak) at beam 512"
+UNIT = "logits/s"
+CFG = 4
+COPIES = 3
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _workload_config(w, extra=None):
+    cfg = {
+        "workload": w.name,
+        "requests": w.R,
+        "beam": w.n,
+        "depth": w.depth,
+        "codes_per_level": w.V,
+        "catalog_sids": w.n_sids,
+        "trie_layout": "dense bitmask levels 1-2, CSR levels 3-5",
+        "logits_dtype": w.dtype,
+        "l2": "inputs larger than L2: 3 rotating copies of the per-step logits (5 steps, 256 MiB + step 0 each)",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, path):
+        self.path = path
+        self.proc = None
+        try:
+            self.f = open(path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        busy = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(busy), "reasons": reasons}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import torch
+
+    import trie_constrained_beam_b200 as tcb
+    from sidgen import device as gdev
+    from sidgen import host
+    from sidgen.workloads import WORKLOADS
+    from trie_constrained_beam_b200 import build as tbuild
+
+    torch.cuda.set_device(local)
+    if rank == 0:
+        tbuild.build()
+        gdev.build()
+    if world > 1:
+        torch.distributed.barrier()
+    w = WORKLOADS[CFG]
+    dev = torch.device("cuda", local)
+    cat = w.catalog()
+    trie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    search = tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth)
+    stream = torch.cuda.current_stream()
+
+    # 1. Generate the search's logits once (generator keyed by prefix hash).
+    hashes = torch.full((w.R,), int(np.uint64(host.PREFIX_HASH_SEED).view(np.int64)),
+                        dtype=torch.int64, device=dev)
+    base = []
+    live_rows = []
+    for t in range(w.depth):
+        rows = search.rows(t)
+        lg = torch.empty((rows, w.V), dtype=torch.bfloat16, device=dev)
+        gdev.row_logits(w.logits_seed, hashes, w.V, w.sigma, lg)
+        ps, pn, B_in = search.parents(t)
+        live_rows.append(int(torch.isfinite(ps).sum().item()))
+        search.step(t, lg)
+        child = torch.empty((w.R * w.n,), dtype=torch.int64, device=dev)
+        gdev.child_hash(hashes, w.R, B_in, search.bp_parent[t], search.bp_code[t], w.n, t + 1, child)
+        hashes = child
+        base.append(lg)
+    search.finalize()
+    ref_sids = search.sids.clone()
+    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+    sets = [base] + [[x.clone() for x in base] for _ in range(args.copies - 1)]
+    torch.cuda.synchronize()
+
+    esize = 2
+    logits_per_search = sum(r * w.V for r in live_rows)
+    mask_row = ((w.V + 31) // 32 + 3) // 4 * 4 * 4
+    step_bytes = []
+    for t in range(w.depth):
+        b = live_rows[t] * w.V * esize + live_rows[t] * 8 + w.R * w.n * 16
+        if w.layouts[t] == 1:
+            b += live_rows[t] * mask_row
+        step_bytes.append(b)
+
+    def one_search(i, ev=None):
+        lset = sets[i % len(sets)]
+        for t in range(w.depth):
+            if ev is not None:
+                ev[t][0].record(stream)
+            search.step(t, lset[t], stream=stream)
+            if ev is not None:
+                ev[t][1].record(stream)
+        search.finalize(stream=stream)
+
+    for i in range(args.warmup):
+        one_search(i)
+    torch.cuda.synchronize()
+    assert torch.equal(search.sids, ref_sids), "replay diverged from the generated search"
+
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in range(w.depth)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, "/tmp/_clk.csv")
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        one_search(i, evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    assert torch.equal(search.sids, ref_sids)
+    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+
+    per_step_us = [statistics.mean(evs[i][t][0].elapsed_time(evs[i][t][1]) for i in range(K)) * 1e3
+                   for t in range(w.depth)]
+    steady = list(range(1, w.depth))
+    dur_us = statistics.mean(per_step_us[t] for t in steady)
+    bytes_launch = statistics.mean(step_bytes[t] for t in steady)
+    peak, peak_kind = _peaks()
+    achieved = bytes_launch / (dur_us * 1e-6) / 1e9
+    value = world * K * logits_per_search / (elapsed_ms * 1e-3)
+
+    # 2. End to end through the C ABI with host buffers: per search, copy every
+    #    step's logits from pinned host memory, run, copy the results back.
+    e2e = None
+    if not args.no_e2e:
+        pinned = [x.cpu().pin_memory() for x in base]
+        dbuf = [torch.empty_like(x) for x in base]
+        out_sids = torch.empty(search.sids.shape, dtype=torch.int32).pin_memory()
+        out_leaf = torch.empty(search.leaf.shape, dtype=torch.int32).pin_memory()
+        out_score = torch.empty((w.R, w.n), dtype=torch.float32).pin_memory()
+        K2 = max(3, min(50, K // 20))
+
+        def e2e_search():
+            for t in range(w.depth):
+                dbuf[t].copy_(pinned[t], non_blocking=True)
+                search.step(t, dbuf[t], stream=stream)
+            sids, leaf, scores = search.finalize(stream=stream)
+            out_sids.copy_(sids, non_blocking=True)
+            out_leaf.copy_(leaf, non_blocking=True)
+            out_score.copy_(scores, non_blocking=True)
+
+        for _ in range(2):
+            e2e_search()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K2):
+            e2e_search()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev)
+            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+            ems = float(tt.item())
+        assert torch.equal(out_sids, ref_sids.cpu())
+        h2d = sum(x.numel() * x.element_size() for x in pinned)
+        d2h = out_sids.numel() * 4 + out_leaf.numel() * 4 + out_score.numel() * 4
+        e2e = {"value": world * K2 * logits_per_search / (ems * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds)
+
+    traffic = _profile_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": _workload_config(w, {"parallelism": f"replicas x{world} (requests sharded)"}),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "beam_step_kernel<bf16>, steady steps 1-4",
+                     "bytes_per_launch": bytes_launch, "us_per_launch": dur_us},
+        "step_us": per_step_us,
+        "logits_per_step": logits_per_search,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "gpu_launches": K * (w.depth + 1),
+    }
+    return line
+
+
+def _profile_traffic():
+    """DRAM bytes per steady beam_step launch from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "beam_step_wide_beam.md")
+    if not os.path.exists(p):
+        return None
+    for ln in open(p):
+        if ln.startswith("traffic_bytes_per_launch:"):
+            try:
+                v = ln.split(":", 1)[1].strip()
+                return None if v in ("", "null") else float(v)
+            except ValueError:
+                return None
+    return None
+
+
+# ----------------------------------------------------------------- oracle timing
+def _oracle_inputs(w, base, search, t):
+    """Host copies of step t's inputs (bf16 bits, parent scores, nodes)."""
+    import torch
+    lg = base[t].view(torch.int16).cpu().numpy().view(np.uint16)
+    ps, pn, B_in = search.parents(t)
+    return lg, ps.cpu().numpy(), pn.cpu().numpy(), B_in
+
+
+def _oracle_trie(w):
+    import oracle
+    return oracle.OracleTrie(w.catalog(), w.codes_per_level)
+
+
+def cpu_baseline(w, base, search, live_rows, budget_s=15.0, trie=None):
+    """Time the oracle's beam step on a bounded sample of steady step 2
+    (whole requests of 512 rows x 4,096 bf16 logits) on this host's cores."""
+    import oracle
+    trie = trie or _oracle_trie(w)
+    t = 2
+    lg, ps, pn, B_in = _oracle_inputs(w, base, search, t)
+    done_rows = 0
+    reqs = 0
+    t0 = time.perf_counter()
+    while reqs < w.R and time.perf_counter() - t0 < budget_s:
+        sl = slice(reqs * B_in, (reqs + 1) * B_in)
+        oracle.beam_step(trie, t, lg[sl], ps[sl], pn[sl], 1, B_in, w.n, w.V)
+        done_rows += int(np.isfinite(ps[sl]).sum())
+        reqs += 1
+    el = time.perf_counter() - t0
+    return {"value": done_rows * w.V / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"oracle.beam_step on {reqs} request(s) of step {t} "
+                      f"({B_in} rows x {w.V} bf16 logits each), {el:.1f} s, numpy float64, "
+                      f"single thread; host has {os.cpu_count()} cores"}
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on bounded samples of
+    the same workload (steady step 2, slices of request 0's rows)."""
+    import oracle
+    from sidgen import host
+    from sidgen.workloads import WORKLOADS
+
+    w = WORKLOADS[CFG]
+    # Inputs of step 2 come from the oracle's own search on host-generated logits
+    # (the oracle needs no GPU): steps 0 and 1 are run once, untimed.
+    trie = _oracle_trie(w)
+
+    def fn(step, prefixes):
+        return host.row_logits(w.logits_seed, host.prefix_hashes(prefixes), w.V, w.sigma, "bf16")
+
+    R1 = 1
+    scores = np.zeros(R1)
+    nodes = np.zeros(R1, dtype=np.int64)
+    prefixes = np.zeros((R1, 1, 0), dtype=np.int64)
+    B_in = 1
+    for t in range(2):
+        z = fn(t, prefixes.reshape(R1 * B_in, t))
+        out = oracle.beam_step(trie, t, z, scores, nodes, R1, B_in, w.n, w.V)
+        newp = np.full((R1, w.n, t + 1), -1, dtype=np.int64)
+        for k in range(w.n):
+            p = out["parent"][0, k]
+            if p >= 0:
+                newp[0, k, :t] = prefixes[0, p]
+                newp[0, k, t] = out["code"][0, k]
+        prefixes, scores, nodes, B_in = newp, out["score"].reshape(-1), out["node"].reshape(-1), w.n
+    t = 2
+    z = fn(t, prefixes.reshape(B_in, t))
+    # Calibrate the per-row cost, then size each step to fit the run in ~2 minutes.
+    c0 = time.perf_counter()
+    oracle.beam_step(trie, t, z[:8], scores[:8], nodes[:8], 1, 8, w.n, w.V)
+    per_row = max((time.perf_counter() - c0) / 8, 1e-5)
+    total_steps = max(1, args.steps + args.warmup)
+    rows_per_step = int(max(1, min(B_in, 120.0 / total_steps / per_row)))
+    pos = 0
+
+    def one():
+        nonlocal pos
+        lo = pos % B_in
+        hi = min(B_in, lo + rows_per_step)
+        oracle.beam_step(trie, t, z[lo:hi], scores[lo:hi], nodes[lo:hi], 1, hi - lo, w.n, w.V)
+        pos = hi % B_in
+        return (hi - lo) * w.V
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        done += one()
+    el = time.perf_counter() - t0
+    value = done / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": _workload_config(w, {"parallelism": "single host thread"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step: oracle.beam_step on {rows_per_step} rows of "
+                                   f"step 2 (x {w.V} bf16 logits), request 0 of the workload"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--copies", type=int, default=COPIES,
+                    help="rotating copies of the per-step logits (3 keeps reads out of L2)")
+    args = ap.parse_args()
+    world, rank, local = _dist()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
