@@ -163,6 +163,33 @@ int beam_step(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dt
               int32_t* out_code, int32_t* out_node, void* workspace, size_t workspace_bytes,
               void* stream);
 
+/* beam_step_noalloc -- the same step as beam_step, for callers that cannot
+ * allocate device memory when they run it (a plugin whose host application owns
+ * every device allocation or enforces a fixed budget, a serving loop that plans
+ * all memory up front and must not call cudaMalloc later). Not in the pages:
+ * it has no counterpart there; it only changes where the scratch space lives.
+ *  Arguments and results are those of beam_step, without the workspace. The
+ *  scratch is a fixed array of SIDBEAM_NOALLOC_SCRATCH_BYTES compiled into the
+ *  library: every GPU that loads the library holds it until the process exits.
+ *  The call allocates nothing. It clears the array's counters on `stream`
+ *  (one memset) and then runs the beam_step kernel on it.
+ *  The first call on each device looks the array's device address up
+ *  (cudaGetSymbolAddress with that device current); make that first call before
+ *  any stream capture.
+ *  All calls share the one array and it keeps the last call's contents: calls
+ *  whose work overlaps on the GPU (other streams, other host threads) race and
+ *  give wrong results; serialise them.
+ *  The device status word also lives in the array and is not reported here.
+ *  Errors: those of beam_step, and WORKSPACE when the shape needs more scratch
+ *  than the array holds (beam_step_workspace_size(R, B_in, n_out, V) >
+ *  SIDBEAM_NOALLOC_SCRATCH_BYTES). */
+#define SIDBEAM_NOALLOC_SCRATCH_BYTES (4 << 20)
+int beam_step_noalloc(const sidbeam_trie* trie, int step, const void* logits,
+                      sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                      const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                      float* out_scores, int32_t* out_parent, int32_t* out_code,
+                      int32_t* out_node, void* stream);
+
 /* beam_finalize -- [P1] Quickstart (beams ranked best-first). Follows the
  * back-pointers of `depth` steps from the last step's ranks.
  *  bp_parent, bp_code device i32 [depth][R][n] (each step's out_parent/out_code).

@@ -41,8 +41,10 @@ EXPORTED = (
     "sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
     "sid_trie_free", "beam_step_workspace_size", "beam_step", "beam_finalize",
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
-    "sidbeam_last_error", "sidbeam_version",
+    "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class SidbeamError(RuntimeError):
@@ -73,6 +75,7 @@ def load():
     L.beam_step_workspace_size.argtypes = [I32, I32, I32, I32]
     L.beam_step_workspace_size.restype = SZ
     L.beam_step.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
+    L.beam_step_noalloc.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P]
     L.beam_finalize.argtypes = [I32, I32, I32, P, P, P, P, P, P]
     L.catalog_score_workspace_size.argtypes = [P, I32, I32]
     L.catalog_score_workspace_size.restype = SZ
@@ -83,7 +86,8 @@ def load():
     L.sidbeam_version.argtypes = []
     L.sidbeam_version.restype = ctypes.c_char_p
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
-                 "beam_step", "beam_finalize", "catalog_score_topk", "sidbeam_get_device_status"):
+                 "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
+                 "sidbeam_get_device_status"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -197,6 +201,20 @@ def beam_step(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V
                           _ptr(out_node), _ptr(workspace),
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
+    _check(rc)
+
+
+def beam_step_noalloc(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V,
+                      out_scores, out_parent, out_code, out_node, stream=None, ld=None):
+    """beam_step with the library's built-in scratch instead of a workspace; for
+    callers that cannot allocate device memory. Calls must not overlap on the GPU."""
+    if ld is None:
+        ld = logits.stride(0)
+    rc = load().beam_step_noalloc(None if trie is None else trie.handle, step, _ptr(logits),
+                                  _dtype_code(logits), ld, _ptr(parent_scores),
+                                  _ptr(parent_nodes), R, B_in, n_out, V, _ptr(out_scores),
+                                  _ptr(out_parent), _ptr(out_code), _ptr(out_node),
+                                  _stream(stream))
     _check(rc)
 
 
