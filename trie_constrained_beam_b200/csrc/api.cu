@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include <cstdio>
 #include <cstring>
 
@@ -83,7 +85,7 @@ extern "C" const char* sidbeam_version(void) { return "0.1.0"; }
 extern "C" size_t beam_step_workspace_size(int R, int B_in, int n_out, int V) {
   if (R < 1 || B_in < 1 || n_out < 1 || n_out > SIDBEAM_MAX_BEAM || V < 1 || V > SIDBEAM_MAX_V)
     return 0;
-  const Partition p = make_partition(R, B_in, device_sm_count());
+  const Partition p = make_partition(R, B_in, std::min(device_sm_count(), 640));
   return workspace_layout(R, p.maxG, n_out).total;
 }
 

@@ -47,6 +47,7 @@ struct ScoreArgs {
   uint32_t* part_count;
   unsigned long long* part_keys;
   int32_t* part_vals;
+  uint32_t* ghist;
   Partition part;
   ScoreConfig cfg;
 };
@@ -62,7 +63,7 @@ struct ScoreWriter {
   }
 };
 
-__global__ void __launch_bounds__(kScoreWarps * 32)
+__global__ void __launch_bounds__(kScoreWarps * 32, 2)
     catalog_score_kernel(const __grid_constant__ ScoreArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const ScoreConfig& cfg = a.cfg;
@@ -80,11 +81,12 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     ctl->abort_flag = 0;
     ctl->counter = 0;
   }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
   WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw, wvals + static_cast<size_t>(warp) * cfg.Cw,
-             whist + warp * 256, cfg.Cw, 0, 0ull};
+             whist + warp * 256, cfg.Cw, 0, 0ull, 0};
   const ScoreWriter writer{a.out_scores, a.out_leaf, a.K};
-  const int64_t row_lo = static_cast<int64_t>(blockIdx.x) * a.part.rows_per_cta;
-  const int64_t row_hi = min(a.part.total_rows, row_lo + a.part.rows_per_cta);
+  int64_t row_lo, row_hi;
+  a.part.range(static_cast<int>(blockIdx.x), row_lo, row_hi);
   const int tsize = a.depth * a.Vmax;
 
   for (int64_t seg_lo = row_lo; seg_lo < row_hi;) {
@@ -94,8 +96,18 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     for (int i = threadIdx.x; i < tsize; i += blockDim.x) table[i] = src[i];
     team_sync(team);
     const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
+    // Histogram reference: the largest possible SID score of this request
+    // (sum over positions of the best code); every warp computes the same value.
+    float C = 0.f;
+    for (int l = 0; l < a.depth; ++l) {
+      float mx = __int_as_float(0xFF800000);
+      for (int c = lane; c < a.Vmax; c += 32) mx = fmaxf(mx, table[l * a.Vmax + c]);
+      C += warp_max(mx);
+    }
+    if (!(C > __int_as_float(0xFF800000) && C < __int_as_float(0x7F800000))) C = 0.f;
     const int64_t j_lo = seg_lo - static_cast<int64_t>(r) * a.N;
     const int64_t j_hi = seg_hi - static_cast<int64_t>(r) * a.N;
+    int batches = 0;
     for (int64_t j0 = j_lo + static_cast<int64_t>(warp) * 32; j0 < j_hi;
          j0 += static_cast<int64_t>(cfg.W) * 32) {
       const int64_t j = j0 + lane;
@@ -106,11 +118,12 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
         for (int l = 1; l < a.depth; ++l)
           score += table[l * a.Vmax + a.leaf_codes[static_cast<int64_t>(l) * a.stride + j]];
       }
-      const unsigned long long cthr =
-          *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
-      if (cthr > wb.thr) wb.thr = cthr;
-      warp_offer(wb, valid, make_key(score, static_cast<uint32_t>(j)), static_cast<int32_t>(j),
-                 static_cast<uint32_t>(a.K), lane, sinks);
+      const uint64_t key = make_key(score, static_cast<uint32_t>(j));
+      const bool pass = valid && key >= wb.thr;
+      if (!__any_sync(0xFFFFFFFFu, pass)) continue;
+      warp_bin(ctl->hist, pass, score_bin(score, C), wb.binned);
+      if ((++batches & 7) == 0) refresh_thr(wb, ctl, static_cast<uint32_t>(a.K), C, lane, sinks);
+      warp_offer(wb, pass, key, static_cast<int32_t>(j), static_cast<uint32_t>(a.K), lane, sinks);
     }
     FlushArgs f;
     f.n = a.K;
@@ -127,7 +140,11 @@ __global__ void __launch_bounds__(kScoreWarps * 32)
     f.cw = cfg.Cw;
     f.sort_keys = wkeys;
     f.sort_vals = wvals;
-    if (segment_flush(team, wb, ctl, cta_hist, f, writer)) return;
+    f.sort_cap = cfg.W * cfg.Cw;
+    f.ghist = a.ghist;
+    f.C = C;
+    f.radix_hist = cta_hist;
+    if (segment_flush(team, wb, ctl, f, writer)) return;
     seg_lo = seg_hi;
   }
 }
@@ -164,6 +181,7 @@ bool choose_score_config(int depth, int Vmax, int K, ScoreConfig* out) {
 }  // namespace sidbeam
 
 using namespace sidbeam;
+using sidbeam::dev::kMaxSegCounts;
 
 static int score_vmax(const sidbeam_trie* t) {
   int v = 1;
@@ -175,7 +193,8 @@ extern "C" size_t catalog_score_workspace_size(const sidbeam_trie* trie, int R, 
   if (!trie || R < 1 || K < 1 || K > SIDBEAM_MAX_BEAM) return 0;
   ScoreConfig cfg;
   if (!choose_score_config(trie->depth, score_vmax(trie), K, &cfg)) return 0;
-  const Partition p = make_partition(R, trie->n_leaves, device_sm_count() * cfg.ctas_per_sm);
+  const Partition p = make_partition(
+      R, trie->n_leaves, std::min(device_sm_count() * cfg.ctas_per_sm, kMaxSegCounts));
   return workspace_layout(R, p.maxG, K).total;
 }
 
@@ -203,7 +222,8 @@ extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, i
   a.K = K;
   a.out_scores = out_scores;
   a.out_leaf = out_leaf;
-  a.part = make_partition(R, trie->n_leaves, device_sm_count() * a.cfg.ctas_per_sm);
+  a.part = make_partition(
+      R, trie->n_leaves, std::min(device_sm_count() * a.cfg.ctas_per_sm, kMaxSegCounts));
   const WorkspaceLayout ws = workspace_layout(R, a.part.maxG, K);
   if (!workspace || workspace_bytes < ws.total)
     return set_error(SIDBEAM_ERR_WORKSPACE, "catalog_score_topk: workspace of %zu bytes, need %zu",
@@ -215,6 +235,7 @@ extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, i
   a.part_count = reinterpret_cast<uint32_t*>(w + ws.part_count);
   a.part_keys = reinterpret_cast<unsigned long long*>(w + ws.part_keys);
   a.part_vals = reinterpret_cast<int32_t*>(w + ws.part_vals);
+  a.ghist = reinterpret_cast<uint32_t*>(w + ws.ghist);
   cudaError_t e = cudaFuncSetAttribute(catalog_score_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        a.cfg.smem_bytes);

@@ -7,7 +7,7 @@
 #include <cstdarg>
 #include <string>
 
-#include "../../include/sidbeam.h"
+#include "sidbeam.h"
 
 namespace sidbeam {
 

@@ -9,24 +9,44 @@
 
 namespace sidbeam {
 
-constexpr int kMaxStepThreads = 288;         // 1 producer + up to 8 consumer warps
+constexpr int kMaxStepThreads = 416;         // 1 producer + up to 12 consumer warps
+constexpr int kMaxStepThreadsReg = 288;      // register-row path: 1 producer + up to 8
 constexpr int kSmemBudget = 232448;          // 227 KiB of dynamic shared memory per CTA
 constexpr int kMaxStages = 32;
 
-// Rows [0, total_rows) in request-major order are cut into `grid` equal
-// chunks of rows_per_cta; the CTAs that touch request r are
-// first_cta(r) .. last_cta(r).
+// Rows [0, total_rows) in request-major order (row = r * B_in + b) are split
+// over CTAs. When there are at least as many CTAs as requests, each request
+// gets its own group of G CTAs (no CTA touches two requests, so no request is
+// merged while other rows of the same CTA still wait); otherwise the rows are
+// cut into equal contiguous chunks that may span request boundaries.
 struct Partition {
   int64_t total_rows;
   int64_t rows_per_cta;
   int grid;
-  int B_in;   // rows per request
-  int maxG;   // upper bound on contributors of any request
+  int B_in;     // rows per request
+  int maxG;     // upper bound on contributors of any request
+  int grouped;  // 1: request r owns CTAs r*G .. r*G+G-1
+  int G;
 
+  __host__ __device__ __forceinline__ void range(int cta, int64_t& lo, int64_t& hi) const {
+    if (grouped) {
+      const int r = cta / G, j = cta - r * G;
+      const int64_t base = static_cast<int64_t>(r) * B_in;
+      lo = base + static_cast<int64_t>(j) * rows_per_cta;
+      hi = lo + rows_per_cta;
+      if (hi > base + B_in) hi = base + B_in;
+    } else {
+      lo = static_cast<int64_t>(cta) * rows_per_cta;
+      hi = lo + rows_per_cta;
+      if (hi > total_rows) hi = total_rows;
+    }
+  }
   __host__ __device__ __forceinline__ int first_cta(int r) const {
+    if (grouped) return r * G;
     return static_cast<int>(static_cast<int64_t>(r) * B_in / rows_per_cta);
   }
   __host__ __device__ __forceinline__ int last_cta(int r) const {
+    if (grouped) return r * G + G - 1;
     return static_cast<int>((static_cast<int64_t>(r + 1) * B_in - 1) / rows_per_cta);
   }
   __host__ __device__ __forceinline__ int contributors(int r) const {
@@ -37,23 +57,39 @@ struct Partition {
 inline Partition make_partition(int R, int64_t B_in, int ctas) {
   Partition p{};
   p.total_rows = static_cast<int64_t>(R) * B_in;
-  int64_t g = ctas < 1 ? 1 : ctas;
+  p.B_in = static_cast<int>(B_in);
+  if (ctas < 1) ctas = 1;
+  if (R <= ctas) {
+    int64_t G = ctas / R;
+    if (G > B_in) G = B_in;
+    if (G < 1) G = 1;
+    p.rows_per_cta = (B_in + G - 1) / G;
+    G = (B_in + p.rows_per_cta - 1) / p.rows_per_cta;
+    p.grouped = 1;
+    p.G = static_cast<int>(G);
+    p.grid = R * p.G;
+    p.maxG = p.G;
+    return p;
+  }
+  int64_t g = ctas;
   if (g > p.total_rows) g = p.total_rows;
   if (g < 1) g = 1;
   p.rows_per_cta = (p.total_rows + g - 1) / g;
   if (p.rows_per_cta < 1) p.rows_per_cta = 1;
   p.grid = static_cast<int>((p.total_rows + p.rows_per_cta - 1) / p.rows_per_cta);
-  p.B_in = static_cast<int>(B_in);
   int64_t mg = (B_in + p.rows_per_cta - 1) / p.rows_per_cta + 1;
   if (mg > p.grid) mg = p.grid;
   p.maxG = static_cast<int>(mg);
+  p.grouped = 0;
+  p.G = 0;
   return p;
 }
 
-// Workspace: [status | tickets[R] | request_thr[R] | part_count[R][maxG] |
-//             part_keys[R][maxG][n] | part_vals[R][maxG][n]], 256-byte aligned parts.
+// Workspace: [status | tickets[R] | request_thr[R] | score histograms[R][1024] |
+//             part_count[R][maxG] | part_keys[R][maxG][n] | part_vals[R][maxG][n]],
+// 256-byte aligned parts. Everything before part_keys must start at zero.
 struct WorkspaceLayout {
-  size_t status, tickets, request_thr, part_count, part_keys, part_vals, total;
+  size_t status, tickets, request_thr, ghist, part_count, part_keys, part_vals, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -67,6 +103,8 @@ inline WorkspaceLayout workspace_layout(int R, int maxG, int n) {
   o = align256(o + static_cast<size_t>(R) * 4);
   w.request_thr = o;
   o = align256(o + static_cast<size_t>(R) * 8);
+  w.ghist = o;
+  o = align256(o + static_cast<size_t>(R) * 1024 * 4);
   w.part_count = o;
   o = align256(o + static_cast<size_t>(R) * maxG * 4);
   w.part_keys = o;
@@ -84,11 +122,15 @@ struct StepConfig {
   int Cw;                 // candidate slots per consumer warp (>= n + 32)
   int stage_bytes;
   int logits_copy_bytes;  // V * sizeof(dtype) rounded up to 16
-  int mask_copy_bytes;    // dense levels: one bitmask row
-  int off_bars, off_ctl, off_meta, off_chist, off_whist, off_stage, off_wkeys, off_wvals;
+  int extra_bytes;        // per stage after the row: dense mask row or staged CSR codes
+  int prefix_words;       // dense levels: per-warp set-bit prefix counts of a mask row
+  int reg;                // rows held in registers (<= 8 KB per row)
+  int off_bars, off_ctl, off_meta, off_chist, off_whist, off_wprefix, off_wmask, off_stage,
+      off_wkeys, off_wvals;
   int smem_bytes;
 };
 
-bool choose_step_config(int V, int esize, int mask_stride_words, int n, StepConfig* cfg);
+bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int n, bool reg,
+                        StepConfig* cfg);
 
 }  // namespace sidbeam

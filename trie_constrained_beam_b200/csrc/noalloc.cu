@@ -16,6 +16,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include <mutex>
 
 #include "internal.h"
@@ -73,7 +75,7 @@ extern "C" int beam_step_noalloc(const sidbeam_trie* trie, int step, const void*
   // The counters at the head of the scratch must start at zero (status word,
   // per-request tickets and bounds, partial-list sizes); clear them on the
   // stream so the call does not depend on what an earlier call left behind.
-  const Partition p = make_partition(R, B_in, device_sm_count());
+  const Partition p = make_partition(R, B_in, std::min(device_sm_count(), 640));
   const WorkspaceLayout ws = workspace_layout(R, p.maxG, n_out);
   const cudaError_t e =
       cudaMemsetAsync(scratch, 0, ws.part_keys, static_cast<cudaStream_t>(stream));

@@ -5,20 +5,32 @@
 // "the n largest keys" is a set with no ties, and "key >= K" for a threshold K
 // found by an MSB-first radix walk selects exactly n of them.
 //
-// Three levels, all exact:
-//  1. warp: candidates above the warp's threshold are appended to a
-//     shared-memory buffer of Cw >= n + 32 entries; when it is full, the warp
-//     finds the n-th largest key K by a radix walk, keeps the n keys >= K and
-//     raises its threshold to K. Any such K is a lower bound on the request's
-//     n-th best key, so it is also published CTA-wide (shared memory) and
-//     request-wide (a global atomicMax) for other warps and CTAs to filter with.
-//  2. CTA (at the end of a request segment): the union of the warp buffers is
-//     cut to its n best, filtered by the request-wide bound, and written to the
-//     CTA's slot of a per-request partial list in global memory.
-//  3. request: the CTA that takes the last ticket of the request (a
-//     threadfence + atomic counter; nothing ever spins) selects the n best of
-//     all partial lists, sorts them (bitonic, descending) and writes them out.
-//     It then zeroes the ticket and the request bound for the next call.
+// Work is cut by thresholds that are always valid lower bounds on the
+// request's n-th best key (there are at least n real candidates at or above
+// them), so filtering by them never drops a member of the top n:
+//  * a score histogram per request: 1024 bins of 1/16 nat below a reference
+//    score C (an upper bound of the request's scores; everything above C falls
+//    in bin 0, everything far below in the last bin). Each CTA keeps one in
+//    shared memory for its current request; candidates are counted before
+//    they are offered, and the first bin whose cumulative count reaches n
+//    gives a threshold one bin further down (so fp32 rounding of the bin index
+//    can never make it too high). At the end of a segment the CTA adds its
+//    counts to the request's global histogram;
+//  * the key at which a warp buffer was compacted (below);
+//  * the largest of these, shared CTA-wide (shared memory) and request-wide
+//    (a global atomicMax).
+// Three levels of exact selection:
+//  1. warp: surviving candidates go to a shared-memory buffer of Cw >= n + 32
+//     entries; when it is full the warp keeps its n best (radix walk) and
+//     raises its threshold to the n-th key;
+//  2. CTA (end of a request segment): entries above the request-wide bound are
+//     cut to the CTA's n best and written to the CTA's slot of the request's
+//     partial lists in global memory;
+//  3. request: the CTA that takes the last ticket (threadfence + atomic
+//     counter; nothing ever spins) reads the complete histogram, copies the
+//     partial entries above its bound into shared memory, selects the n best,
+//     sorts them (bitonic, descending), writes them out and zeroes the ticket,
+//     bound and histogram for the next call.
 #pragma once
 
 #include "device_utils.cuh"
@@ -27,7 +39,9 @@ namespace sidbeam {
 namespace dev {
 
 constexpr int kBarConsumers = 1;  // named barrier id used by the consumer warps
-constexpr int kMaxSegCounts = 1024;
+constexpr int kMaxSegCounts = 640;
+constexpr int kHistBins = 1024;
+constexpr float kHistScale = 16.f;  // bins per nat
 
 // The consumer warps of a CTA (the threads that run selection).
 struct Team {
@@ -55,6 +69,7 @@ __device__ __forceinline__ bool team_sync_or(const Team& t, bool pred) {
   return res != 0;
 }
 
+// ------------------------------------------------------------ radix select
 // Given a 256-bin histogram of the current digit (only bins < 2^width are
 // non-zero), finds digit d such that the keys in higher bins number `above`
 // < need <= above + hist[d]. Warp-collective (one warp).
@@ -101,10 +116,23 @@ __device__ __forceinline__ void find_digit_warp(const uint32_t* hist, uint32_t n
   cnt = __shfl_sync(0xFFFFFFFFu, ct, src);
 }
 
+// Histogram increment (shared-memory atomic). Lanes with `active` false add
+// nothing; lanes may call it divergently.
+__device__ __forceinline__ void hist_add(uint32_t* hist, bool active, uint32_t bin, int) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
+
+// Score-histogram increment by a whole warp; counts the additions for the
+// refresh policy. Warp-collective.
+__device__ __forceinline__ void warp_bin(uint32_t* hist, bool active, uint32_t bin, int& binned) {
+  if (active) atomicAdd(&hist[bin], 1u);
+  binned += __popc(__ballot_sync(0xFFFFFFFFu, active));
+}
+
 // Threshold K with exactly `need` keys >= K among keys[0..count) (count > need >= 1).
 // Warp-collective; hist = 256 words of this warp's shared memory.
-__device__ inline uint64_t warp_select(const uint64_t* keys, int count, uint32_t need, uint32_t* hist,
-                                int lane) {
+__device__ inline uint64_t warp_select(const uint64_t* keys, int count, uint32_t need,
+                                       uint32_t* hist, int lane) {
   uint64_t a = ~0ull, o = 0;
   for (int i = lane; i < count; i += 32) {
     const uint64_t k = keys[i];
@@ -122,10 +150,11 @@ __device__ inline uint64_t warp_select(const uint64_t* keys, int count, uint32_t
     const uint32_t dmask = (1u << (hi - lo)) - 1u;
     for (int i = lane; i < 256; i += 32) hist[i] = 0;
     __syncwarp();
-    for (int i = lane; i < count; i += 32) {
-      const uint64_t k = keys[i];
-      const bool match = hi >= 64 || ((k >> hi) == (prefix >> hi));
-      if (match) atomicAdd(&hist[static_cast<uint32_t>(k >> lo) & dmask], 1u);
+    for (int base = 0; base < count; base += 32) {
+      const int i = base + lane;
+      const uint64_t k = i < count ? keys[i] : 0ull;
+      const bool match = i < count && (hi >= 64 || ((k >> hi) == (prefix >> hi)));
+      hist_add(hist, match, static_cast<uint32_t>(k >> lo) & dmask, lane);
     }
     __syncwarp();
     int d;
@@ -139,7 +168,65 @@ __device__ inline uint64_t warp_select(const uint64_t* keys, int count, uint32_t
   }
 }
 
-// Shared-memory control block of the selection (one per CTA).
+// ------------------------------------------------------------ score histogram
+__device__ __forceinline__ uint32_t score_bin(float score, float C) {
+  const float x = (C - score) * kHistScale;
+  if (!(x >= 0.f)) return 0u;  // above the reference (or NaN reference)
+  if (x >= static_cast<float>(kHistBins - 1)) return kHistBins - 1;
+  return static_cast<uint32_t>(x);
+}
+
+// Smallest key of any candidate whose score is >= s (its score half only).
+__device__ __forceinline__ uint64_t key_floor(float s) {
+  return static_cast<uint64_t>(ord_f32(s)) << 32;
+}
+
+// From a histogram with at least n counted candidates in bins 0..k, those
+// candidates all score above C - (k+2)/16 (one bin of slack for fp32 rounding
+// of the bin index), so key_floor of that value is a valid lower bound.
+// Returns 0 when fewer than n are counted or the bound falls in the last bins.
+// Warp-collective over a 1024-bin, 16-byte aligned histogram.
+__device__ __forceinline__ uint64_t hist_bound(const uint32_t* hist, uint32_t n, float C,
+                                               int lane) {
+  // Lane l owns bins 32l .. 32l+31; its eight 16-byte reads are rotated by l
+  // so that the 8 lanes of each access phase hit 8 different bank groups.
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist) + lane * 8;
+  uint32_t s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint4 v = h4[(j + lane) & 7];
+    s += v.x + v.y + v.z + v.w;
+  }
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned b = __ballot_sync(0xFFFFFFFFu, incl >= n);
+  if (b == 0) return 0ull;
+  const int src = __ffs(b) - 1;
+  int k = 0;
+  if (lane == src) {  // one lane walks its own 32 bins in order
+    uint32_t cum = incl - s;
+    int j = 0;
+    for (; j < 7; ++j) {
+      const uint4 v = h4[j];
+      const uint32_t c = v.x + v.y + v.z + v.w;
+      if (cum + c >= n) break;
+      cum += c;
+    }
+    const uint32_t* hb = hist + lane * 32 + j * 4;
+    int e = 0;
+    while (e < 3 && cum + hb[e] < n) cum += hb[e++];
+    k = lane * 32 + j * 4 + e;
+  }
+  k = __shfl_sync(0xFFFFFFFFu, k, src);
+  if (k >= kHistBins - 2) return 0ull;
+  return key_floor(C - static_cast<float>(k + 2) / kHistScale);
+}
+
+// ------------------------------------------------------------ shared control
 struct SelCtl {
   unsigned long long cta_thr;  // CTA-wide lower bound on the segment's n-th best key
   unsigned long long bcast_key;
@@ -150,25 +237,31 @@ struct SelCtl {
   int counter;
   int is_last;
   int abort_flag;
+  int staged;
+  int next_item;               // dynamic ring-item claims (beam_step)
   int wcount[32];
-  int segcnt[kMaxSegCounts];
+  int segoff[kMaxSegCounts + 1];
+  __align__(16) uint32_t hist[kHistBins];  // score histogram of the current segment
 };
 
-// Key sources for the CTA-level select.
+// Key source for the CTA-level select: nseg buffers of stride cw.
 struct WarpBufSrc {
-  const uint64_t* keys;  // [nwarps][cw]
+  const uint64_t* keys;  // [nseg][cw]
   int cw;
   const int* counts;     // shared
   int nseg;
   __device__ __forceinline__ int count(int s) const { return counts[s]; }
   __device__ __forceinline__ uint64_t key(int s, int i) const { return keys[s * cw + i]; }
 };
+
+// Key source for the CTA-level select: one request's partial lists in global
+// memory (list k holds segoff[k+1] - segoff[k] entries at stride n).
 struct PartialSrc {
-  const unsigned long long* keys;  // partial lists of one request: [maxG][n]
+  const unsigned long long* keys;
   int n;
-  const int* counts;               // shared copy of the list sizes
+  const int* segoff;  // shared
   int nseg;
-  __device__ __forceinline__ int count(int s) const { return counts[s]; }
+  __device__ __forceinline__ int count(int s) const { return segoff[s + 1] - segoff[s]; }
   __device__ __forceinline__ uint64_t key(int s, int i) const {
     return __ldcg(keys + static_cast<size_t>(s) * n + i);
   }
@@ -176,6 +269,7 @@ struct PartialSrc {
 
 // CTA-level threshold: K with exactly `need` keys >= K over all segments of src
 // (total > need >= 1). All consumer threads call it; uses team_sync.
+// `hist` is a 256-word scratch histogram.
 template <class Src>
 __device__ uint64_t cta_select(const Team& t, const Src& src, uint32_t need, uint32_t* hist,
                                SelCtl* ctl) {
@@ -212,10 +306,11 @@ __device__ uint64_t cta_select(const Team& t, const Src& src, uint32_t need, uin
     team_sync(t);
     for (int s = 0; s < src.nseg; ++s) {
       const int c = src.count(s);
-      for (int i = t.tid; i < c; i += t.T) {
-        const uint64_t k = src.key(s, i);
-        const bool match = hi >= 64 || ((k >> hi) == (prefix >> hi));
-        if (match) atomicAdd(&hist[static_cast<uint32_t>(k >> lo) & dmask], 1u);
+      for (int base = 0; base < c; base += t.T) {
+        const int i = base + t.tid;
+        const uint64_t k = i < c ? src.key(s, i) : 0ull;
+        const bool match = i < c && (hi >= 64 || ((k >> hi) == (prefix >> hi)));
+        hist_add(hist, match, static_cast<uint32_t>(k >> lo) & dmask, t.lane);
       }
     }
     team_sync(t);
@@ -241,10 +336,45 @@ __device__ uint64_t cta_select(const Team& t, const Src& src, uint32_t need, uin
 }
 
 // Bitonic sort of N (a power of two) (key, value) pairs in shared memory into
-// descending key order.
+// descending key order. Compare-exchanges whose partners lie within one
+// aligned block of 32 run inside a warp on registers (shuffles); only strides
+// of 32 and more go through shared memory with a barrier per stride.
+__device__ __forceinline__ void bitonic_warp_block(const Team& t, uint64_t* keys, int32_t* vals,
+                                                   int N, int size_lo, int size_hi,
+                                                   int first_stride) {
+  for (int blk = t.warp; blk * 32 < N; blk += t.nwarps) {
+    const int i = blk * 32 + t.lane;
+    const bool in = i < N;
+    uint64_t k = in ? keys[i] : 0ull;
+    int32_t v = in ? vals[i] : -1;
+    for (int size = size_lo; size <= size_hi; size <<= 1) {
+      const int s0 = size == size_lo ? first_stride : (size >> 1);
+      for (int stride = s0; stride > 0; stride >>= 1) {
+        const uint64_t pk = __shfl_xor_sync(0xFFFFFFFFu, k, stride);
+        const int32_t pv = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+        const bool lower = (t.lane & stride) == 0;
+        const bool desc = (i & size) == 0;
+        const bool take = (lower == desc) ? (pk > k) : (pk < k);
+        if (take) {
+          k = pk;
+          v = pv;
+        }
+      }
+    }
+    if (in) {
+      keys[i] = k;
+      vals[i] = v;
+    }
+  }
+}
+
 __device__ inline void cta_bitonic_desc(const Team& t, uint64_t* keys, int32_t* vals, int N) {
-  for (int size = 2; size <= N; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+  if (N < 2) return;
+  // Sizes 2 .. min(N, 32): entirely inside warps.
+  bitonic_warp_block(t, keys, vals, N, 2, N < 32 ? N : 32, 1);
+  team_sync(t);
+  for (int size = 64; size <= N; size <<= 1) {
+    for (int stride = size >> 1; stride >= 32; stride >>= 1) {
       for (int i = t.tid; i < (N >> 1); i += t.T) {
         const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
         const int hi = lo + stride;
@@ -260,24 +390,37 @@ __device__ inline void cta_bitonic_desc(const Team& t, uint64_t* keys, int32_t* 
       }
       team_sync(t);
     }
+    bitonic_warp_block(t, keys, vals, N, size, size, 16);
+    team_sync(t);
   }
 }
 
-// Per-warp candidate buffer.
+// ------------------------------------------------------------ warp buffers
 struct WarpBuf {
   uint64_t* keys;   // [cw] shared
   int32_t* vals;    // [cw] shared
-  uint32_t* hist;   // [256] shared
+  uint32_t* hist;   // [256] shared, radix-select scratch
   int cw;
   int count;        // warp-uniform
   uint64_t thr;     // warp-uniform: candidates need key >= thr
+  int binned;       // warp-uniform: candidates counted in the CTA histogram since the last refresh
 };
+
+// Candidates counted by this warp in the CTA histogram before it rescans it.
+constexpr int kRefreshAfter = 32;
 
 // Where a warp publishes its thresholds.
 struct ThrSinks {
   unsigned long long* cta_thr;     // shared
   unsigned long long* request_thr; // global, may be null
 };
+
+__device__ __forceinline__ void publish_thr(uint64_t K, int lane, const ThrSinks& sinks) {
+  if (lane == 0) {
+    atomicMax(sinks.cta_thr, static_cast<unsigned long long>(K));
+    if (sinks.request_thr) atomicMax(sinks.request_thr, static_cast<unsigned long long>(K));
+  }
+}
 
 // Keep the n best of the buffer (count > n), raise and publish the threshold.
 __device__ __forceinline__ void warp_compact(WarpBuf& wb, uint32_t n, int lane,
@@ -303,13 +446,9 @@ __device__ __forceinline__ void warp_compact(WarpBuf& wb, uint32_t n, int lane,
   }
   wb.count = out;
   if (K > wb.thr) wb.thr = K;
-  if (lane == 0) {
-    atomicMax(sinks.cta_thr, static_cast<unsigned long long>(K));
-    if (sinks.request_thr) atomicMax(sinks.request_thr, static_cast<unsigned long long>(K));
-  }
+  publish_thr(K, lane, sinks);
   __syncwarp();
 }
-
 
 // Offer one candidate per lane (only lanes with valid = true). Warp-collective:
 // every lane of the warp must call it with the same wb state.
@@ -333,6 +472,29 @@ __device__ __forceinline__ void warp_offer(WarpBuf& wb, bool valid, uint64_t key
   wb.count += cnt;
 }
 
+// Raise the warp threshold from the CTA histogram and the CTA-wide bound
+// (the request-wide bound is read once per row by the caller, not here, to
+// keep an L2 round trip off this path). Warp-collective.
+__device__ __forceinline__ void refresh_thr(WarpBuf& wb, SelCtl* ctl, uint32_t n, float C,
+                                            int lane, const ThrSinks& sinks) {
+  if (wb.binned < kRefreshAfter && wb.thr != 0ull) {
+    const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+    if (c > wb.thr) wb.thr = c;
+    return;
+  }
+  wb.binned = 0;
+  const uint64_t hb = hist_bound(ctl->hist, n, C, lane);
+  const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+  uint64_t t = wb.thr;
+  if (c > t) t = c;
+  if (hb > t) {
+    t = hb;
+    publish_thr(hb, lane, sinks);
+  }
+  wb.thr = t;
+}
+
+// ------------------------------------------------------------ segment end
 // Everything a CTA needs to hand its segment of request r over.
 struct FlushArgs {
   int n;                  // beams (or K) to select per request
@@ -345,100 +507,297 @@ struct FlushArgs {
   uint32_t* part_count;           // [R][maxG]
   uint32_t* tickets;              // [R]
   unsigned long long* request_thr;  // [R]
+  uint32_t* ghist;                // [R][kHistBins]
+  float C;                        // histogram reference score of request r
   const uint64_t* wkeys;  // all warp buffers, [nwarps][cw]
   int cw;
   uint64_t* sort_keys;    // shared scratch for the final sort (aliases the warp buffers)
   int32_t* sort_vals;
+  int sort_cap;           // entries available at sort_keys / sort_vals
+  uint32_t* radix_hist;   // 256-word scratch for cta_select
 };
 
-// The last contributor of request r: select the n best of all partial lists,
-// sort them and hand each rank to `out(r, rank, key, val, valid)`.
+// Warp-aggregated append position: this lane's slot among the `keep` lanes.
+__device__ __forceinline__ int append_pos(int* counter, bool keep, int lane) {
+  const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
+  int base = 0;
+  if (lane == 0 && bal) base = atomicAdd(counter, __popc(bal));
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  return base + __popc(bal & lanemask_lt());
+}
+
+// The last contributor of request r: bound from the complete histogram, copy
+// the partial entries above it into shared memory, select the n best, sort
+// them and hand each rank to `out(r, rank, key, val, valid)`.
 template <class Writer>
-__device__ void request_merge(const Team& t, SelCtl* ctl, uint32_t* hist, const FlushArgs& f,
-                              const Writer& out) {
+__device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, const Writer& out) {
   const int G = f.G < kMaxSegCounts ? f.G : kMaxSegCounts;
   const size_t list0 = static_cast<size_t>(f.r) * f.maxG;
+  // The CTA histogram area now receives the request's complete histogram.
+  uint32_t* gh = f.ghist + static_cast<size_t>(f.r) * kHistBins;
+  for (int i = t.tid; i < kHistBins; i += t.T) ctl->hist[i] = __ldcg(gh + i);
   for (int k = t.tid; k < G; k += t.T) {
     const int c = static_cast<int>(__ldcg(f.part_count + list0 + k));
-    ctl->segcnt[k] = c < f.n ? c : f.n;
+    ctl->segoff[k + 1] = c < f.n ? c : f.n;
   }
   team_sync(t);
-  int M = 0;
-  for (int k = 0; k < G; ++k) M += ctl->segcnt[k];
+  if (t.warp == 0) {  // exclusive prefix sum of the list sizes
+    int carry = 0;
+    for (int k0 = 0; k0 < G; k0 += 32) {
+      const int k = k0 + t.lane;
+      const int c = k < G ? ctl->segoff[k + 1] : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (t.lane >= o) incl += y;
+      }
+      if (k < G) ctl->segoff[k + 1] = carry + incl;
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (t.lane == 0) {
+      ctl->segoff[0] = 0;
+      ctl->counter = 0;
+    }
+  }
+  team_sync(t);
+  if (t.warp == 0) {
+    const uint64_t hb = hist_bound(ctl->hist, static_cast<uint32_t>(f.n), f.C, t.lane);
+    if (t.lane == 0) {
+      const unsigned long long g =
+          *reinterpret_cast<volatile unsigned long long*>(f.request_thr + f.r);
+      ctl->bcast_key = hb > g ? hb : g;
+    }
+  }
+  team_sync(t);
+  const uint64_t K0 = ctl->bcast_key;
+  const int total = ctl->segoff[G];
   const unsigned long long* lists = f.part_keys + list0 * f.n;
   const int32_t* lvals = f.part_vals + list0 * f.n;
-  uint64_t K = 0;
-  if (M > f.n) K = cta_select(t, PartialSrc{lists, f.n, ctl->segcnt, G}, f.n, hist, ctl);
-  const int sel = M < f.n ? M : f.n;
-  int N = 1;
-  while (N < sel) N <<= 1;
-  for (int i = t.tid; i < N; i += t.T) {
-    f.sort_keys[i] = 0ull;
-    f.sort_vals[i] = -1;
-  }
-  if (t.tid == 0) ctl->counter = 0;
-  team_sync(t);
-  for (int k = 0; k < G; ++k) {
-    const int c = ctl->segcnt[k];
-    for (int i = t.tid; i < c; i += t.T) {
-      const uint64_t key = __ldcg(lists + static_cast<size_t>(k) * f.n + i);
-      if (key >= K) {
-        const int pos = atomicAdd(&ctl->counter, 1);
-        if (pos < N) {
-          f.sort_keys[pos] = key;
-          f.sort_vals[pos] = __ldcg(lvals + static_cast<size_t>(k) * f.n + i);
+  // Filtered copy of all partial entries >= K0 into [0, cap): flat index,
+  // segment found by binary search, four independent loads per thread.
+  uint64_t* stk = f.sort_keys;
+  int32_t* stv = f.sort_vals;
+  const int cap = f.sort_cap;
+  for (int base = 0; base < total; base += 4 * t.T) {
+    uint64_t key[4];
+    int32_t val[4];
+    bool in[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = base + u * t.T + t.tid;
+      in[u] = i < total;
+      key[u] = 0ull;
+      val[u] = -1;
+      if (in[u]) {
+        int lo = 0, hi = G;  // segoff[lo] <= i < segoff[hi]
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (ctl->segoff[mid] <= i) lo = mid; else hi = mid;
         }
+        const size_t at = static_cast<size_t>(lo) * f.n + (i - ctl->segoff[lo]);
+        key[u] = __ldcg(lists + at);
+        val[u] = __ldcg(lvals + at);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool keep = in[u] && key[u] >= K0 && key[u] != 0ull;
+      const int pos = append_pos(&ctl->counter, keep, t.lane);
+      if (keep && pos < cap) {
+        stk[pos] = key[u];
+        stv[pos] = val[u];
       }
     }
   }
   team_sync(t);
-  cta_bitonic_desc(t, f.sort_keys, f.sort_vals, N);
+  int M = ctl->counter;
+  if (M > cap) {
+    // The bound left more entries than shared memory holds (a poor histogram
+    // reference): select straight from the lists in L2 instead.
+    M = total;
+    const int sel_all = M < f.n ? M : f.n;
+    int N_all = 1;
+    while (N_all < sel_all) N_all <<= 1;
+    uint64_t Kg = 0;
+    if (M > f.n)
+      Kg = cta_select(t, PartialSrc{lists, f.n, ctl->segoff, G}, f.n, f.radix_hist, ctl);
+    if (t.tid == 0) ctl->counter = 0;
+    for (int i = t.tid; i < N_all; i += t.T) {
+      stk[i] = 0ull;
+      stv[i] = -1;
+    }
+    team_sync(t);
+    for (int base = 0; base < total; base += t.T) {
+      const int i = base + t.tid;
+      uint64_t key = 0ull;
+      int32_t val = -1;
+      if (i < total) {
+        int lo = 0, hi = G;
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (ctl->segoff[mid] <= i) lo = mid; else hi = mid;
+        }
+        const size_t at = static_cast<size_t>(lo) * f.n + (i - ctl->segoff[lo]);
+        key = __ldcg(lists + at);
+        val = __ldcg(lvals + at);
+      }
+      const bool keep = i < total && key >= Kg && key != 0ull;
+      const int pos = append_pos(&ctl->counter, keep, t.lane);
+      if (keep && pos < N_all) {
+        stk[pos] = key;
+        stv[pos] = val;
+      }
+    }
+    team_sync(t);
+    cta_bitonic_desc(t, stk, stv, N_all);
+    for (int i = t.tid; i < f.n; i += t.T) {
+      const bool valid = i < sel_all;
+      out(f.r, i, valid ? stk[i] : 0ull, valid ? stv[i] : -1, valid);
+    }
+    for (int i = t.tid; i < kHistBins; i += t.T) gh[i] = 0u;
+    if (t.tid == 0) {
+      f.tickets[f.r] = 0u;
+      f.request_thr[f.r] = 0ull;
+    }
+    return;
+  }
+  const int sel = M < f.n ? M : f.n;
+  int N = 1;
+  while (N < sel) N <<= 1;
+  uint64_t K = 0;
+  if (M > f.n) {
+    if (t.tid == 0) ctl->staged = M;
+    team_sync(t);
+    K = cta_select(t, WarpBufSrc{stk, 0, &ctl->staged, 1}, f.n, f.radix_hist, ctl);
+  }
+  // Sort buffer: behind the staged entries if they fit, else the staged entries
+  // themselves (keys below K zeroed: they sort last).
+  uint64_t* sk = stk;
+  int32_t* sv = stv;
+  const int m32 = (M + 31) & ~31;
+  if (M > f.n && m32 + N <= cap) {
+    sk = stk + m32;
+    sv = stv + m32;
+    if (t.tid == 0) ctl->counter = 0;
+    for (int i = t.tid; i < N; i += t.T) {
+      sk[i] = 0ull;
+      sv[i] = -1;
+    }
+    team_sync(t);
+    for (int base = 0; base < M; base += t.T) {
+      const int i = base + t.tid;
+      const bool keep = i < M && stk[i] >= K;
+      const int pos = append_pos(&ctl->counter, keep, t.lane);
+      if (keep && pos < N) {
+        sk[pos] = stk[i];
+        sv[pos] = stv[i];
+      }
+    }
+  } else {
+    const int span = N > M ? N : M;
+    for (int i = t.tid; i < span; i += t.T) {
+      if (i >= M || stk[i] < K) {
+        stk[i] = 0ull;
+        stv[i] = -1;
+      }
+    }
+  }
+  team_sync(t);
+  if (sk == stk && M > N) {
+    // Entries above K are scattered over [0, M): pack them into [0, N) first.
+    // (Only reached when the staging area had no room for a second buffer.)
+    if (t.tid == 0) {
+      int w = 0;
+      for (int i = 0; i < M; ++i)
+        if (stk[i] != 0ull) {
+          stk[w] = stk[i];
+          stv[w] = stv[i];
+          ++w;
+        }
+      for (int i = w; i < M; ++i) {
+        stk[i] = 0ull;
+        stv[i] = -1;
+      }
+    }
+    team_sync(t);
+  }
+  cta_bitonic_desc(t, sk, sv, N);
+  const uint64_t* ok_keys = sk;
+  const int32_t* ok_vals = sv;
   for (int i = t.tid; i < f.n; i += t.T) {
     const bool valid = i < sel;
-    out(f.r, i, valid ? f.sort_keys[i] : 0ull, valid ? f.sort_vals[i] : -1, valid);
+    out(f.r, i, valid ? ok_keys[i] : 0ull, valid ? ok_vals[i] : -1, valid);
+  }
+  // Leave the request's histogram, ticket and bound zeroed for the next call.
+  for (int i = t.tid; i < kHistBins; i += t.T) gh[i] = 0u;
+  if (t.tid == 0) {
+    f.tickets[f.r] = 0u;
+    f.request_thr[f.r] = 0ull;
   }
 }
 
 // End of a request segment for this CTA (all consumer warps call it).
 // Returns true when the CTA must stop (an abort was seen by any warp).
 template <class Writer>
-__device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, uint32_t* hist,
-                              const FlushArgs& f, const Writer& out) {
+__device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const FlushArgs& f,
+                              const Writer& out) {
   if (t.lane == 0) ctl->wcount[t.warp] = wb.count;
   if (team_sync_or(t, ctl->abort_flag != 0)) return true;
-  int total = 0;
-  for (int w = 0; w < t.nwarps; ++w) total += ctl->wcount[w];
-  uint64_t K = 0;
-  if (total > f.n)
-    K = cta_select(t, WarpBufSrc{f.wkeys, f.cw, ctl->wcount, t.nwarps}, f.n, hist, ctl);
-  if (t.tid == 0) {
-    unsigned long long old;
-    if (total > f.n)
-      old = atomicMax(f.request_thr + f.r, static_cast<unsigned long long>(K));
-    else
-      old = *reinterpret_cast<volatile unsigned long long*>(f.request_thr + f.r);
-    ctl->bcast_key = old > K ? old : K;
-    ctl->counter = 0;
+  // 1. Add this segment's histogram to the request's (read back only by the
+  //    merging CTA); bound the flush by this CTA's histogram and the shared bounds.
+  uint32_t* gh = f.ghist + static_cast<size_t>(f.r) * kHistBins;
+  for (int i = t.tid; i < kHistBins; i += t.T) {
+    const uint32_t c = ctl->hist[i];
+    if (c) atomicAdd(gh + i, c);
+  }
+  if (t.warp == 0) {
+    const uint64_t hb = hist_bound(ctl->hist, static_cast<uint32_t>(f.n), f.C, t.lane);
+    if (t.lane == 0) {
+      const unsigned long long g =
+          *reinterpret_cast<volatile unsigned long long*>(f.request_thr + f.r);
+      const unsigned long long c = ctl->cta_thr;
+      unsigned long long K = hb;
+      if (g > K) K = g;
+      if (c > K) K = c;
+      ctl->bcast_key = K;
+      ctl->counter = 0;
+    }
   }
   team_sync(t);
-  K = ctl->bcast_key;
+  uint64_t K = ctl->bcast_key;
+  // 2. Entries above the bound; cut to the CTA's n best if there are more.
+  {
+    int ge = 0;
+    for (int base = 0; base < wb.count; base += 32) {
+      const int i = base + t.lane;
+      ge += __popc(__ballot_sync(0xFFFFFFFFu, i < wb.count && wb.keys[i] >= K));
+    }
+    if (t.lane == 0 && ge) atomicAdd(&ctl->counter, ge);
+  }
+  team_sync(t);
+  if (ctl->counter > f.n) {
+    const uint64_t Kc = cta_select(t, WarpBufSrc{f.wkeys, f.cw, ctl->wcount, t.nwarps}, f.n,
+                                   f.radix_hist, ctl);
+    if (Kc > K) K = Kc;
+    if (t.tid == 0) atomicMax(f.request_thr + f.r, static_cast<unsigned long long>(K));
+  }
+  team_sync(t);
+  if (t.tid == 0) ctl->counter = 0;
+  team_sync(t);
   const size_t slot = (static_cast<size_t>(f.r) * f.maxG + f.k) * f.n;
   for (int base = 0; base < wb.count; base += 32) {
     const int i = base + t.lane;
     const bool keep = i < wb.count && wb.keys[i] >= K;
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, keep);
-    int pos0 = 0;
-    if (t.lane == 0 && bal) pos0 = atomicAdd(&ctl->counter, __popc(bal));
-    pos0 = __shfl_sync(0xFFFFFFFFu, pos0, 0);
-    if (keep) {
-      const int pos = pos0 + __popc(bal & lanemask_lt());
-      if (pos < f.n) {
-        f.part_keys[slot + pos] = wb.keys[i];
-        f.part_vals[slot + pos] = wb.vals[i];
-      }
+    const int pos = append_pos(&ctl->counter, keep, t.lane);
+    if (keep && pos < f.n) {
+      f.part_keys[slot + pos] = wb.keys[i];
+      f.part_vals[slot + pos] = wb.vals[i];
     }
   }
+  __threadfence();  // every thread's histogram adds and list writes, before the ticket
   team_sync(t);
+  // 3. Ticket; the last contributor merges the request.
   if (t.tid == 0) {
     const int c = ctl->counter < f.n ? ctl->counter : f.n;
     f.part_count[static_cast<size_t>(f.r) * f.maxG + f.k] = static_cast<uint32_t>(c);
@@ -449,12 +808,11 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, uint32_t*
   team_sync(t);
   if (ctl->is_last) {
     __threadfence();
-    request_merge(t, ctl, hist, f, out);
-    if (t.tid == 0) {
-      f.tickets[f.r] = 0u;
-      f.request_thr[f.r] = 0ull;
-    }
+    request_merge(t, ctl, f, out);
+    team_sync(t);
   }
+  // 4. Reset for the next segment.
+  for (int i = t.tid; i < kHistBins; i += t.T) ctl->hist[i] = 0u;
   wb.count = 0;
   wb.thr = 0;
   if (t.tid == 0) ctl->cta_thr = 0ull;
