@@ -5,23 +5,27 @@
 // Features > Serving ("API"): deterministic top-k at temperature 0.
 //
 // Design (sm_100a):
-//  * One CTA per SM. Rows are split evenly over CTAs; a CTA's rows may span
-//    request boundaries (one "segment" per request it touches).
-//  * Warp 0 is the producer: it reads each row's parent score / node and, for
-//    live rows only, issues untiled bulk copies (cp.async.bulk, TMA engine) of
-//    the logits row and of the node's trie data -- the bitmask row at dense
-//    levels, the child-code range at CSR levels -- into a ring of S
-//    shared-memory stages that complete on mbarriers.
-//  * Warps 1..W are consumers. They claim ring items in order. A row of up to
-//    8 KB is copied into registers together with what the candidate walk needs
-//    from the stage, and the stage goes back to the producer at once; larger
-//    rows are worked on in place. The row max and sum of exp over the FULL
-//    codebook give lse = m + log(sum) (fp32, packed f32x2 arithmetic, warp
-//    shuffles); then the node's children are walked twice: first counted in
-//    the CTA's score histogram, then, above the raised threshold, offered as
-//    key(score = s + (z_c - lse), idx = b*V + c) to the warp's top-n buffer.
-//  * At the end of each segment the consumer warps run the CTA merge and, in
-//    the last contributing CTA of the request, the request merge (topn.cuh).
+//  * One CTA per SM; the rows of a CTA are dealt to its warps (row i of the
+//    CTA to warp i mod W). When a CTA has fewer rows than warps, every warp
+//    takes every row and the candidate walk is split between them.
+//  * Every warp streams its own rows: it owns a ring of S shared-memory
+//    stages and, from one lane, issues untiled bulk copies (cp.async.bulk,
+//    the TMA engine; no multicast) of the logits row and of the node's trie
+//    data (the dense bitmask row, or the first child codes at CSR levels)
+//    into a stage that completes on the stage's mbarrier. The first copies go
+//    out before the row's parent score and node have even been read.
+//  * A row of up to 8 KB is copied into registers (plus the trie data its
+//    candidate walk needs) and the stage is refilled at once with the warp's
+//    row S places ahead; larger rows are worked on in place.
+//  * Row max and the full-codebook log-normaliser lse = m + log(sum exp(z-m))
+//    in fp32 (packed f32x2 arithmetic, ex2.approx, warp shuffles); then the
+//    node's children are walked twice, above a threshold that is always a
+//    valid lower bound on the request's n-th best key: first counted in the
+//    CTA's score histogram, then offered as key(score = s + (z_c - lse),
+//    idx = b*V + c) to the warp's top-n buffer.
+//  * At the end of a request segment the warps hand their candidates over
+//    (topn.cuh): a CTA that holds a whole request ranks them itself, else the
+//    last of the request's CTAs ranks everyone's partial lists.
 // The logits are read exactly once from HBM.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -41,11 +45,10 @@ using namespace dev;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRegVecs = 16;  // 16-byte vectors per lane held in registers (8 KB rows)
-
-enum ItemKind : int32_t { kItemRow = 0, kItemSegmentEnd = 1, kItemExit = 2 };
+constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // f(I) for I = 0 .. N-1 with I a compile-time constant (keeps register arrays
-// indexed statically even where the compiler would not unroll a loop).
+// indexed statically).
 template <int I> struct Idx { static constexpr int value = I; };
 template <int N>
 struct Unrolled {
@@ -60,45 +63,6 @@ struct Unrolled<0> {
   template <class F>
   __device__ __forceinline__ static void run(F&&) {}
 };
-
-struct __align__(16) Meta {
-  int32_t kind;
-  int32_t req;
-  int64_t row;
-  float score;     // parent score s
-  int32_t node;    // parent node p
-  uint32_t o0;     // children of p: ids o0 .. o1-1
-  uint32_t o1;
-  uint32_t seq;    // ring item number; written before the full-barrier arrive
-  uint32_t a0;     // CSR: first staged child id (o0 rounded down to a multiple of 8)
-  uint32_t nst;    // CSR: child codes staged from a0 on
-  float C;         // histogram reference of the row's request
-};
-
-// Consumer-side wait for ring item `item` in `stage`. Several consumer warps
-// share the ring, so a warp can reach a stage while the previous item there
-// (another warp's) is still in flight; an mbarrier parity wait would then
-// match the older phase. Waiting first for the producer to publish this
-// item's number makes the stage's pending phase the item's own, after which
-// the parity wait is exact. Both waits are bounded.
-__device__ __forceinline__ bool wait_item(const Meta* meta, uint64_t* full, int stage,
-                                          uint32_t item, uint32_t S, volatile int* abort_flag,
-                                          uint32_t* status) {
-  const volatile uint32_t* seqp = &meta[stage].seq;
-  if (*seqp != item) {
-    const uint64_t t0 = global_timer_ns();
-    while (*seqp != item) {
-      __nanosleep(64);
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        atomicOr(status, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-  return bounded_wait(&full[stage], (item / S) & 1u, abort_flag, status, kStatusTimeout);
-}
 
 struct StepArgs {
   const uint8_t* logits;
@@ -127,8 +91,7 @@ struct StepArgs {
   uint32_t* ghist;
   Partition part;
   StepConfig cfg;
-  int coop;     // 1: every consumer warp works on every row (few rows per CTA)
-  int markers;  // segment-end / exit markers per event: W (claimed) or 1 (coop)
+  int coop;  // 1: every warp takes every row of the CTA (fewer rows than warps)
 };
 
 struct StepWriter {
@@ -288,29 +251,6 @@ __device__ __forceinline__ float vec_elem(const uint4& x, int j) {
   return __uint_as_float(w);
 }
 
-// x[k] for a warp-uniform runtime k, through constant indices only (a
-// register array indexed at run time would be moved to local memory).
-__device__ __forceinline__ uint4 pick_vec(const uint4 (&x)[kRegVecs], int k) {
-  switch (k) {
-    case 0: return x[0];
-    case 1: return x[1];
-    case 2: return x[2];
-    case 3: return x[3];
-    case 4: return x[4];
-    case 5: return x[5];
-    case 6: return x[6];
-    case 7: return x[7];
-    case 8: return x[8];
-    case 9: return x[9];
-    case 10: return x[10];
-    case 11: return x[11];
-    case 12: return x[12];
-    case 13: return x[13];
-    case 14: return x[14];
-    default: return x[15];
-  }
-}
-
 // Elements j >= keep of a vector become -inf (they lie past V).
 __device__ __forceinline__ uint32_t cut_word_bf16(uint32_t w, int first, int keep) {
   if (first >= keep) return 0xFF80FF80u;
@@ -373,153 +313,6 @@ __device__ __forceinline__ void row_stats_reg(const uint4 (&x)[kRegVecs], int nv
   lse_out = m + logf(sum);
 }
 
-// --------------------------------------------------------------- producer
-// Histogram reference of request r: its first parent's score (an upper bound
-// of every child score when parents arrive ranked best-first, as beam_step
-// writes them); any finite value keeps the histogram bounds valid.
-__device__ __forceinline__ float request_ref(const StepArgs& a, int r) {
-  const float c = a.parent_scores[static_cast<int64_t>(r) * a.B_in];
-  return (c > __int_as_float(0xFF800000) && c < __int_as_float(0x7F800000)) ? c : 0.f;
-}
-
-__device__ void producer(const StepArgs& a, uint8_t* stages, Meta* meta, uint64_t* full,
-                         uint64_t* empty, SelCtl* ctl, int64_t row_lo, int64_t row_hi, int lane) {
-  const StepConfig& cfg = a.cfg;
-  const int S = cfg.S;
-  const uint64_t pol = policy_evict_first();
-  const uint32_t max_codes = static_cast<uint32_t>(cfg.extra_bytes / 2);
-  uint32_t item = 0;
-  bool ok = true;
-
-  auto acquire = [&](uint32_t it) -> int {
-    const int stage = static_cast<int>(it % S);
-    if (it >= static_cast<uint32_t>(S)) {
-      const uint32_t parity = ((it / S) - 1) & 1u;
-      if (!bounded_wait(&empty[stage], parity, &ctl->abort_flag, a.status, kStatusTimeout))
-        return -1;
-    }
-    return stage;
-  };
-
-  int64_t seg_lo = row_lo;
-  while (ok && seg_lo < row_hi) {
-    const int r = static_cast<int>(seg_lo / a.B_in);
-    const int64_t seg_hi = min(row_hi, static_cast<int64_t>(r + 1) * a.B_in);
-    const float C = request_ref(a, r);
-    for (int64_t base = seg_lo; ok && base < seg_hi; base += 32) {
-      const int64_t row = base + lane;
-      const bool in = row < seg_hi;
-      float s = __int_as_float(0xFF800000);
-      int32_t p = -1;
-      if (in) {
-        s = a.parent_scores[row];
-        p = a.layout ? a.parent_nodes[row] : 0;
-      }
-      bool live = in && s != __int_as_float(0xFF800000);
-      if (a.layout) {
-        if (p < 0) {
-          live = false;
-        } else if (static_cast<int64_t>(p) >= a.n_parent) {
-          if (live) atomicOr(a.status, kStatusBadNode);
-          live = false;
-        }
-      }
-      uint32_t o0 = 0, o1 = 0;
-      if (live && a.layout) {
-        o0 = a.off[p];
-        o1 = a.off[p + 1];
-      }
-      unsigned lm = __ballot_sync(0xFFFFFFFFu, live);
-      while (lm) {
-        const int j = __ffs(lm) - 1;
-        lm &= lm - 1;
-        const float sj = __shfl_sync(0xFFFFFFFFu, s, j);
-        const int32_t pj = __shfl_sync(0xFFFFFFFFu, p, j);
-        const uint32_t o0j = __shfl_sync(0xFFFFFFFFu, o0, j);
-        const uint32_t o1j = __shfl_sync(0xFFFFFFFFu, o1, j);
-        const int stage = acquire(item);
-        if (stage < 0) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          Meta& m = meta[stage];
-          m.kind = kItemRow;
-          m.req = r;
-          m.row = base + j;
-          m.score = sj;
-          m.node = pj;
-          m.o0 = o0j;
-          m.o1 = o1j;
-          m.C = C;
-          uint8_t* dst = stages + static_cast<size_t>(stage) * cfg.stage_bytes;
-          uint32_t extra = 0;
-          uint32_t a0 = o0j & ~7u, nst = 0;
-          if (a.layout == SIDBEAM_LAYOUT_DENSE) {
-            extra = static_cast<uint32_t>(cfg.extra_bytes);
-          } else if (a.layout == SIDBEAM_LAYOUT_CSR && o1j > o0j) {
-            nst = min(o1j - a0, max_codes);
-            extra = (nst * 2 + 15) & ~15u;
-          }
-          m.a0 = a0;
-          m.nst = nst;
-          m.seq = item;
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(cfg.logits_copy_bytes) + extra);
-          bulk_copy_g2s(dst, a.logits + (base + j) * a.row_bytes,
-                        static_cast<uint32_t>(cfg.logits_copy_bytes), &full[stage], pol);
-          if (a.layout == SIDBEAM_LAYOUT_DENSE)
-            bulk_copy_g2s(dst + cfg.logits_copy_bytes,
-                          a.mask + static_cast<size_t>(pj) * a.mask_stride, extra, &full[stage],
-                          pol);
-          else if (extra)
-            bulk_copy_g2s(dst + cfg.logits_copy_bytes, a.codes + a0, extra, &full[stage], pol);
-        }
-        __syncwarp();
-        ++item;
-      }
-    }
-    // One segment-end marker per consumer warp (claimed in order, so each warp
-    // gets exactly one); in cooperative mode every warp reads every item.
-    for (int w = 0; ok && w < a.markers; ++w) {
-      const int stage = acquire(item);
-      if (stage < 0) {
-        ok = false;
-        break;
-      }
-      if (lane == 0) {
-        meta[stage].kind = kItemSegmentEnd;
-        meta[stage].req = r;
-        meta[stage].C = C;
-        meta[stage].seq = item;
-        mbar_arrive(&full[stage]);
-      }
-      __syncwarp();
-      ++item;
-    }
-    seg_lo = seg_hi;
-  }
-  for (int w = 0; ok && w < a.markers; ++w) {
-    const int stage = acquire(item);
-    if (stage < 0) {
-      ok = false;
-      break;
-    }
-    if (lane == 0) {
-      meta[stage].kind = kItemExit;
-      meta[stage].seq = item;
-      mbar_arrive(&full[stage]);
-    }
-    __syncwarp();
-    ++item;
-  }
-  if (!ok) {
-    // Abort: let the copies already issued land before the CTA exits.
-    const uint32_t first = item > static_cast<uint32_t>(S) ? item - S : 0u;
-    for (uint32_t it = first; it < item; ++it) drain_wait(&full[it % S], (it / S) & 1u);
-  }
-}
-
-// --------------------------------------------------------------- consumers
 // Node id of dense child code c: first child id + rank of c among the node's
 // set bits. `prefix` holds the set-bit counts before each mask word.
 __device__ __forceinline__ int32_t dense_child(const uint32_t* mrow, const uint32_t* prefix,
@@ -547,74 +340,329 @@ __device__ __forceinline__ void dense_prefix(const uint32_t* mrow, int words, ui
   __syncwarp();
 }
 
+
+// --------------------------------------------------------------- warp rings
+// The rows a warp takes, in order: row(i) for i < count.
+struct RowSeq {
+  int64_t first;
+  int64_t stride;
+  int count;
+  __device__ __forceinline__ int64_t row(int i) const { return first + stride * i; }
+};
+
+// Parent data of 32 consecutive entries of a warp's row sequence, one per lane.
+struct MetaBatch {
+  int base;         // sequence index of lane 0's row (a multiple of 32)
+  float s;          // parent score
+  int32_t p;        // parent node
+  uint32_t o0, o1;  // children of p: ids o0 .. o1-1 (trie levels only)
+  unsigned live;    // lanes whose row is expanded
+};
+
+// A row is dead (skipped, its logits never used) when its parent score is
+// -inf or, with a trie, its node is negative; a node past the level's end is
+// also skipped and reported in the status word.
+__device__ __forceinline__ void load_meta(const StepArgs& a, const RowSeq& q, int base, int lane,
+                                          MetaBatch& m) {
+  const int i = base + lane;
+  const bool in = i < q.count;
+  float s = __int_as_float(0xFF800000);
+  int32_t p = -1;
+  if (in) {
+    const int64_t row = q.row(i);
+    s = a.parent_scores[row];
+    p = a.layout ? a.parent_nodes[row] : 0;
+  }
+  bool live = in && s != __int_as_float(0xFF800000);
+  if (a.layout) {
+    if (p < 0) {
+      live = false;
+    } else if (static_cast<int64_t>(p) >= a.n_parent) {
+      if (live) atomicOr(a.status, kStatusBadNode);
+      live = false;
+    }
+  }
+  uint32_t o0 = 0, o1 = 0;
+  if (live && a.layout) {
+    o0 = a.off[p];
+    o1 = a.off[p + 1];
+  }
+  m.base = base;
+  m.s = s;
+  m.p = p;
+  m.o0 = o0;
+  m.o1 = o1;
+  m.live = __ballot_sync(kFull, live);
+}
+
+// CSR: child codes staged behind the row start at id a0 = o0 rounded down to
+// a multiple of 8 (a 16-byte boundary); at most extra_bytes / 2 of them.
+__device__ __forceinline__ uint32_t csr_staged(const StepArgs& a, uint32_t o0, uint32_t o1) {
+  if (o1 <= o0) return 0u;
+  const uint32_t n = o1 - (o0 & ~7u);
+  const uint32_t cap = static_cast<uint32_t>(a.cfg.extra_bytes / 2);
+  return n < cap ? n : cap;
+}
+
+// Bytes of trie data staged behind a live row.
+__device__ __forceinline__ uint32_t extra_bytes(const StepArgs& a, uint32_t o0, uint32_t o1) {
+  if (a.layout == SIDBEAM_LAYOUT_DENSE) return static_cast<uint32_t>(a.mask_stride) * 4u;
+  if (a.layout == SIDBEAM_LAYOUT_CSR) return (csr_staged(a, o0, o1) * 2u + 15u) & ~15u;
+  return 0u;
+}
+
+// Copy of the trie data of node p behind the row (one lane; bytes > 0).
+__device__ __forceinline__ void copy_extra(const StepArgs& a, uint8_t* stage, uint64_t* bar,
+                                           int32_t p, uint32_t o0, uint32_t bytes,
+                                           uint64_t pol) {
+  const void* src = a.layout == SIDBEAM_LAYOUT_DENSE
+                        ? static_cast<const void*>(a.mask + static_cast<size_t>(p) * a.mask_stride)
+                        : static_cast<const void*>(a.codes + (o0 & ~7u));
+  bulk_copy_g2s(stage + a.cfg.logits_copy_bytes, src, bytes, bar, pol);
+}
+
+// One warp's ring. Entry k of the warp's ring traffic goes to stage k % S; the
+// parent data of the row in stage j is kept in lane j (st_*).
+struct Ring {
+  uint8_t* stages;
+  uint64_t* full;
+  int S;
+  int consumed;  // rows taken out of the ring (warp-uniform)
+  int issued;    // rows put into the ring (warp-uniform)
+  int ip;        // next sequence index to look at for issuing (warp-uniform)
+  int st_seq;
+  int st_live;
+  float st_s;
+  int32_t st_p;
+  uint32_t st_o0, st_o1;
+};
+
+// Puts the next live row of the sequence into the stage just released (the
+// ring is full whenever this succeeds, so that stage is issued % S). The
+// stage's earlier contents were read by this warp's lanes: __syncwarp orders
+// those reads before lane 0, and the proxy fence before the async copy.
+// Returns false when the sequence has no live row left. Warp-collective.
+__device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, MetaBatch& mb,
+                                           Ring& g, int lane, uint64_t pol) {
+  while (g.ip < q.count) {
+    if (g.ip >= mb.base + 32) load_meta(a, q, g.ip & ~31, lane, mb);
+    const unsigned m = mb.live & (~0u << (g.ip - mb.base));
+    if (m == 0u) {
+      g.ip = mb.base + 32;
+      continue;
+    }
+    const int j = __ffs(m) - 1;
+    const float s = __shfl_sync(kFull, mb.s, j);
+    const int32_t p = __shfl_sync(kFull, mb.p, j);
+    const uint32_t o0 = __shfl_sync(kFull, mb.o0, j);
+    const uint32_t o1 = __shfl_sync(kFull, mb.o1, j);
+    const int seq = mb.base + j;
+    const int stage = g.issued % g.S;
+    if (lane == stage) {
+      g.st_seq = seq;
+      g.st_live = 1;
+      g.st_s = s;
+      g.st_p = p;
+      g.st_o0 = o0;
+      g.st_o1 = o1;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      uint8_t* dst = g.stages + static_cast<size_t>(stage) * a.cfg.stage_bytes;
+      const uint32_t ex = extra_bytes(a, o0, o1);
+      mbar_arrive_expect_tx(&g.full[stage], static_cast<uint32_t>(a.cfg.logits_copy_bytes) + ex);
+      bulk_copy_g2s(dst, a.logits + q.row(seq) * a.row_bytes,
+                    static_cast<uint32_t>(a.cfg.logits_copy_bytes), &g.full[stage], pol);
+      if (ex) copy_extra(a, dst, &g.full[stage], p, o0, ex, pol);
+    }
+    g.ip = seq + 1;
+    ++g.issued;
+    return true;
+  }
+  return false;
+}
+
+// --------------------------------------------------------------- row walks
+// What the walks need to know about a row.
+struct RowCtx {
+  float s;        // parent score
+  float lse;      // log-normaliser over the full codebook
+  float C;        // histogram reference of the request
+  uint32_t idx0;  // b * V (key index of code 0)
+  uint32_t o0;    // first child id
+  uint32_t o1;    // one past the last child id
+};
+
 // Code of CSR child id k: from the stage when it was staged, else from HBM/L2.
-__device__ __forceinline__ int csr_code(const StepArgs& a, const uint8_t* zrow, const Meta& m,
-                                        uint32_t k) {
-  const uint32_t i = k - m.a0;
-  if (i < m.nst) return reinterpret_cast<const uint16_t*>(zrow + a.cfg.logits_copy_bytes)[i];
+__device__ __forceinline__ int csr_code(const StepArgs& a, const uint8_t* zrow, uint32_t o0,
+                                        uint32_t nst, uint32_t k) {
+  const uint32_t i = k - (o0 & ~7u);
+  if (i < nst) return reinterpret_cast<const uint16_t*>(zrow + a.cfg.logits_copy_bytes)[i];
   return a.codes[k];
 }
 
-// Threshold state at the start of a row.
+// Warp threshold at the start of a row: the CTA-wide and request-wide bounds.
 __device__ __forceinline__ void row_thresholds(WarpBuf& wb, SelCtl* ctl, unsigned long long req) {
   const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
   if (c > wb.thr) wb.thr = c;
   if (req > wb.thr) wb.thr = req;
 }
 
-// Row worked on in place in its stage (rows over 8 KB, or CSR rows with more
-// children than one 32-lane batch per warp). The caller returns the stage.
+// Copies a row of up to 8 KB from its stage into registers (vector lane + 32k
+// in x[k]); entries past V become -inf.
 template <int BF16>
-__device__ __forceinline__ void process_row_smem(const StepArgs& a, const uint8_t* zrow, const Meta& m,
-                                 WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix, int lane, int part,
-                                 int nparts) {
+__device__ __forceinline__ void copy_row_regs(const uint8_t* zrow, int V, int lane,
+                                              uint4 (&x)[kRegVecs]) {
   constexpr int kPerVec = BF16 ? 8 : 4;
-  const int r = m.req;
-  const uint32_t b = static_cast<uint32_t>(m.row - static_cast<int64_t>(r) * a.B_in);
-  const uint32_t idx0 = b * static_cast<uint32_t>(a.V);
-  const float s = m.score;
-  const float C = m.C;
-  const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
-  const unsigned long long req_thr =
-      *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+  const int nvec = (V + kPerVec - 1) / kPerVec;
+  const uint4* q = reinterpret_cast<const uint4*>(zrow);
+  const uint4 ninf = BF16 ? make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u)
+                          : make_uint4(0xFF800000u, 0xFF800000u, 0xFF800000u, 0xFF800000u);
+  if (nvec == 32 * kRegVecs && V % kPerVec == 0) {  // a full 8 KB row: plain loads
+    Unrolled<kRegVecs>::run([&](auto kc) {
+      constexpr int k = decltype(kc)::value;
+      x[k] = q[lane + 32 * k];
+    });
+    return;
+  }
+  const int tail = V % kPerVec;
+  const int vt = tail ? nvec - 1 : -1;
+  Unrolled<kRegVecs>::run([&](auto kc) {
+    constexpr int k = decltype(kc)::value;
+    const int v = lane + 32 * k;
+    x[k] = v < nvec ? q[v] : ninf;
+    if (v == vt) vec_cut<BF16>(x[k], tail);
+  });
+}
 
-  float rmax, lse;
-  row_stats<BF16>(zrow, a.V, lane, rmax, lse);
-  row_thresholds(wb, ctl, req_thr);
-  float zthr = zthreshold(wb.thr, s, lse);
+// x[k] for a warp-uniform runtime k, through constant indices only (a
+// register array indexed at run time would be moved to local memory).
+__device__ __forceinline__ uint4 pick_vec(const uint4 (&x)[kRegVecs], int k) {
+  switch (k) {
+    case 0: return x[0];
+    case 1: return x[1];
+    case 2: return x[2];
+    case 3: return x[3];
+    case 4: return x[4];
+    case 5: return x[5];
+    case 6: return x[6];
+    case 7: return x[7];
+    case 8: return x[8];
+    case 9: return x[9];
+    case 10: return x[10];
+    case 11: return x[11];
+    case 12: return x[12];
+    case 13: return x[13];
+    case 14: return x[14];
+    default: return x[15];
+  }
+}
+
+// Bit k set: this lane's vector k (lane + 32k) is this warp's to walk and its
+// largest logit reaches the threshold.
+template <int BF16>
+__device__ __forceinline__ uint32_t vec_flags(const uint4 (&x)[kRegVecs], int nvec, float zthr,
+                                              int lane, int part, int nparts) {
+  uint32_t f = 0u;
+  Unrolled<kRegVecs>::run([&](auto kc) {
+    constexpr int k = decltype(kc)::value;
+    if (32 * k < nvec && (k % nparts) == part && lane + 32 * k < nvec &&
+        vec_max<BF16>(x[k]) >= zthr)
+      f |= 1u << k;
+  });
+  return f;
+}
+
+// One walk over the flagged vectors of a register row at a dense level or
+// without a trie. PASS 0 counts the children at or above the threshold in the
+// CTA histogram; PASS 1 offers them (re-testing each vector against the
+// raised threshold). The loop runs over vectors flagged in any lane.
+template <int BF16, int PASS>
+__device__ __forceinline__ void reg_extract(const StepArgs& a, const uint4 (&x)[kRegVecs],
+                                            uint32_t flags, const uint32_t* wmask,
+                                            uint32_t* wprefix, bool& have_prefix,
+                                            const RowCtx& c, float& zthr, WarpBuf& wb,
+                                            SelCtl* ctl, const ThrSinks& sinks, int lane) {
+  constexpr int kPerVec = BF16 ? 8 : 4;
+  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
+  uint32_t todo = __reduce_or_sync(kFull, flags);
+  while (todo) {
+    const int k = __ffs(todo) - 1;
+    todo &= todo - 1u;
+    const uint4 xk = pick_vec(x, k);
+    const int v = lane + 32 * k;
+    unsigned bits = 0u;
+    if (((flags >> k) & 1u) && (PASS == 0 || vec_max<BF16>(xk) >= zthr)) {
+      const int cb = v * kPerVec;
+      unsigned valid = (1u << kPerVec) - 1u;
+      if (dense)
+        valid = BF16 ? static_cast<unsigned>(reinterpret_cast<const uint8_t*>(wmask)[v])
+                     : (wmask[v >> 3] >> ((v & 7) * 4)) & 0xFu;
+      if (a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+#pragma unroll
+      for (int j = 0; j < kPerVec; ++j)
+        if (((valid >> j) & 1u) && vec_elem<BF16>(xk, j) >= zthr) bits |= 1u << j;
+    }
+    while (__any_sync(kFull, bits != 0u)) {
+      const bool has = bits != 0u;
+      const int j = has ? __ffs(bits) - 1 : 0;
+      bits &= bits - 1u;
+      const int code = v * kPerVec + j;
+      const float score = c.s + (vec_elem<BF16>(xk, j) - c.lse);
+      if (PASS == 0) {
+        warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned);
+      } else {
+        if (dense && !have_prefix) {
+          dense_prefix(wmask, a.mask_words, wprefix, lane);
+          have_prefix = true;
+        }
+        const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code) : -1;
+        warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
+                      static_cast<uint32_t>(a.n), lane, sinks);
+      }
+    }
+    if (PASS == 1) zthr = zthreshold(wb.thr, c.s, c.lse);
+  }
+}
+
+// Candidate walks of a row in place in its stage (rows over 8 KB, or CSR rows
+// with more children than one 32-lane batch per warp).
+template <int BF16>
+__device__ void smem_walks(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
+                           float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
+                           const ThrSinks& sinks, int lane, int part, int nparts) {
+  constexpr int kPerVec = BF16 ? 8 : 4;
   if (rmax < zthr) return;  // even the row's largest logit cannot reach the threshold
-
   if (a.layout == SIDBEAM_LAYOUT_CSR) {
+    const uint32_t nst = csr_staged(a, c.o0, c.o1);
     const uint32_t k_step = static_cast<uint32_t>(32 * nparts);
-    const uint32_t k_begin = m.o0 + static_cast<uint32_t>(part * 32);
+    const uint32_t k_begin = c.o0 + static_cast<uint32_t>(part * 32);
     for (int pass = 0; pass < 2; ++pass) {
-      for (uint32_t k0 = k_begin; k0 < m.o1; k0 += k_step) {
+      for (uint32_t k0 = k_begin; k0 < c.o1; k0 += k_step) {
         const uint32_t k = k0 + lane;
-        const bool in = k < m.o1;
-        const int c = in ? csr_code(a, zrow, m, k) : 0;
-        const float z = in ? elem<BF16>(zrow, c) : 0.f;
+        const bool in = k < c.o1;
+        const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
+        const float z = in ? elem<BF16>(zrow, code) : 0.f;
         const bool ok = in && z >= zthr;
-        if (!__any_sync(0xFFFFFFFFu, ok)) continue;
-        const float score = s + (z - lse);
+        if (!__any_sync(kFull, ok)) continue;
+        const float score = c.s + (z - c.lse);
         if (pass == 0) {
-          warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned);
+          warp_bin(ctl->hist, ok, score_bin(score, c.C), wb.binned);
         } else {
-          warp_offer(wb, ok, make_key(score, idx0 + static_cast<uint32_t>(c)),
-                     static_cast<int32_t>(k), a.n, lane, sinks);
-          zthr = zthreshold(wb.thr, s, lse);
+          warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(code)),
+                        static_cast<int32_t>(k), static_cast<uint32_t>(a.n), lane, sinks);
+          zthr = zthreshold(wb.thr, c.s, c.lse);
         }
       }
       if (pass == 0) {
         __syncwarp();
-        refresh_thr(wb, ctl, a.n, C, lane, sinks);
-        zthr = zthreshold(wb.thr, s, lse);
+        refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), c.C, lane, sinks);
+        zthr = zthreshold(wb.thr, c.s, c.lse);
       }
     }
     return;
   }
-
-  // Dense bitmask or no trie: walk 16-byte vectors; a vector is opened only if
-  // its largest logit reaches the threshold.
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
   const uint32_t* mrow = reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes);
   const int nvec_all = (a.V + kPerVec - 1) / kPerVec;
@@ -623,7 +671,7 @@ __device__ __forceinline__ void process_row_smem(const StepArgs& a, const uint8_
   for (int pass = 0; pass < 2; ++pass) {
     for (int v0 = part * 32; v0 < nvec_all; v0 += 32 * nparts) {
       const int v = v0 + lane;
-      unsigned bits = 0;
+      unsigned bits = 0u;
       if (v < nvec_all) {
         const uint4 x = q[v];
         if (vec_max<BF16>(x) >= zthr) {
@@ -635,174 +683,64 @@ __device__ __forceinline__ void process_row_smem(const StepArgs& a, const uint8_
               bits |= 1u << j;
         }
       }
-      if (!__any_sync(0xFFFFFFFFu, bits != 0u)) continue;
+      if (!__any_sync(kFull, bits != 0u)) continue;
       if (pass == 1 && dense && !have_prefix) {
         dense_prefix(mrow, a.mask_words, wprefix, lane);
         have_prefix = true;
       }
-      while (__any_sync(0xFFFFFFFFu, bits != 0u)) {
+      while (__any_sync(kFull, bits != 0u)) {
         const bool has = bits != 0u;
         const int j = has ? __ffs(bits) - 1 : 0;
         bits &= bits - 1u;
-        const int c = v * kPerVec + j;
-        const float score = has ? s + (elem<BF16>(zrow, c) - lse) : 0.f;
+        const int code = v * kPerVec + j;
+        const float score = has ? c.s + (elem<BF16>(zrow, code) - c.lse) : 0.f;
         if (pass == 0) {
-          warp_bin(ctl->hist, has, score_bin(score, C), wb.binned);
+          warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned);
         } else {
-          const int32_t node = (has && dense) ? dense_child(mrow, wprefix, m.o0, c) : -1;
-          warp_offer(wb, has, make_key(score, idx0 + static_cast<uint32_t>(c)), node, a.n, lane,
-                     sinks);
+          const int32_t node = (has && dense) ? dense_child(mrow, wprefix, c.o0, code) : -1;
+          warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
+                        static_cast<uint32_t>(a.n), lane, sinks);
         }
       }
-      if (pass == 1) zthr = zthreshold(wb.thr, s, lse);
+      if (pass == 1) zthr = zthreshold(wb.thr, c.s, c.lse);
     }
     if (pass == 0) {
       __syncwarp();
-      refresh_thr(wb, ctl, a.n, C, lane, sinks);
-      zthr = zthreshold(wb.thr, s, lse);
+      refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), c.C, lane, sinks);
+      zthr = zthreshold(wb.thr, c.s, c.lse);
     }
   }
 }
 
-// Row of up to 8 KB: copied into registers (plus the trie data the candidate
-// walk needs: the dense mask row into warp-private shared memory, or this
-// lane's CSR child), then the stage is returned before any arithmetic.
-template <int BF16>
-__device__ __forceinline__ void process_row_reg(const StepArgs& a, const uint8_t* zrow, uint64_t* empty_bar,
-                                const Meta& m, WarpBuf& wb, SelCtl* ctl, uint32_t* wmask,
-                                uint32_t* wprefix, int lane, int part, int nparts) {
-  constexpr int kPerVec = BF16 ? 8 : 4;
-  const int V = a.V;
-  const int nvec = (V + kPerVec - 1) / kPerVec;
-  const int r = m.req;
-  const uint32_t b = static_cast<uint32_t>(m.row - static_cast<int64_t>(r) * a.B_in);
-  const uint32_t idx0 = b * static_cast<uint32_t>(V);
-  const float s = m.score;
-  const float C = m.C;
-  const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
-  const unsigned long long req_thr =
-      *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
-  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
-
-  const uint4* q = reinterpret_cast<const uint4*>(zrow);
-  const uint4 ninf = BF16 ? make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u)
-                          : make_uint4(0xFF800000u, 0xFF800000u, 0xFF800000u, 0xFF800000u);
-  uint4 x[kRegVecs];
-  const int tail = V % kPerVec;
-  const int vt = tail ? nvec - 1 : -1;
-  Unrolled<kRegVecs>::run([&](auto kc) {
-    constexpr int k = decltype(kc)::value;
-    const int v = lane + 32 * k;
-    x[k] = v < nvec ? q[v] : ninf;
-    if (v == vt) vec_cut<BF16>(x[k], tail);
-  });
-  if (dense) {
-    const uint32_t* mrow = reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes);
-    for (int i = lane; i < a.mask_stride; i += 32) wmask[i] = mrow[i];
+// Histogram reference of request r: the largest finite parent score of the
+// request (every child score is at most its parent's score), the same value
+// in every CTA. Two slots alternate so that one can be cleared while the
+// other is read. All team threads call it.
+__device__ __forceinline__ float segment_ref(const StepArgs& a, const Team& t, SelCtl* ctl, int r,
+                                             int slot) {
+  float m = __int_as_float(0xFF800000);
+  const float* ps = a.parent_scores + static_cast<int64_t>(r) * a.B_in;
+  for (int i = t.tid; i < a.B_in; i += t.T) {
+    const float x = ps[i];
+    if (x > __int_as_float(0xFF800000) && x < __int_as_float(0x7F800000)) m = fmaxf(m, x);
   }
-  const uint32_t ck = m.o0 + static_cast<uint32_t>(part * 32 + lane);
-  const bool cin = csr && ck < m.o1;
-  int ccode = 0;
-  float cz = 0.f;
-  if (cin) {
-    ccode = csr_code(a, zrow, m, ck);
-    cz = elem<BF16>(zrow, ccode);
-  }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(empty_bar);  // the producer may refill the stage now
-
-  float rmax, lse;
-  row_stats_reg<BF16>(x, nvec, lane, rmax, lse);
-  row_thresholds(wb, ctl, req_thr);
-  float zthr = zthreshold(wb.thr, s, lse);
-  if (rmax < zthr) return;
-
-  if (csr) {
-    for (int pass = 0; pass < 2; ++pass) {
-      const bool ok = cin && cz >= zthr;
-      if (__any_sync(0xFFFFFFFFu, ok)) {
-        const float score = s + (cz - lse);
-        if (pass == 0) {
-          warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned);
-          __syncwarp();
-          refresh_thr(wb, ctl, a.n, C, lane, sinks);
-          zthr = zthreshold(wb.thr, s, lse);
-        } else {
-          warp_offer(wb, ok, make_key(score, idx0 + static_cast<uint32_t>(ccode)),
-                     static_cast<int32_t>(ck), a.n, lane, sinks);
-        }
-      } else {
-        break;
-      }
-    }
-    return;
-  }
-
-  bool have_prefix = false;
-  for (int pass = 0; pass < 2; ++pass) {
-    // Which of this lane's vectors can hold a child above the threshold.
-    uint32_t flags = 0;
-    Unrolled<kRegVecs>::run([&](auto kc) {
-      constexpr int k = decltype(kc)::value;
-      if (32 * k < nvec && (k % nparts) == part && lane + 32 * k < nvec &&
-          vec_max<BF16>(x[k]) >= zthr)
-        flags |= 1u << k;
-    });
-    uint32_t todo = __reduce_or_sync(0xFFFFFFFFu, flags);
-    while (todo) {
-      const int k = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const uint4 xk = pick_vec(x, k);
-      const int v = lane + 32 * k;
-      unsigned bits = 0;
-      if ((flags >> k) & 1u) {
-        const int cb = v * kPerVec;
-        unsigned valid = (1u << kPerVec) - 1u;
-        if (dense) valid = (wmask[cb >> 5] >> (cb & 31)) & ((1u << kPerVec) - 1u);
-#pragma unroll
-        for (int j = 0; j < kPerVec; ++j)
-          if (((valid >> j) & 1u) && cb + j < V && vec_elem<BF16>(xk, j) >= zthr)
-            bits |= 1u << j;
-      }
-      if (!__any_sync(0xFFFFFFFFu, bits != 0u)) continue;
-      if (pass == 1 && dense && !have_prefix) {
-        dense_prefix(wmask, a.mask_words, wprefix, lane);
-        have_prefix = true;
-      }
-      while (__any_sync(0xFFFFFFFFu, bits != 0u)) {
-        const bool has = bits != 0u;
-        const int j = has ? __ffs(bits) - 1 : 0;
-        bits &= bits - 1u;
-        const int c = v * kPerVec + j;
-        const float score = has ? s + (vec_elem<BF16>(xk, j) - lse) : 0.f;
-        if (pass == 0) {
-          warp_bin(ctl->hist, has, score_bin(score, C), wb.binned);
-        } else {
-          const int32_t node = (has && dense) ? dense_child(wmask, wprefix, m.o0, c) : -1;
-          warp_offer(wb, has, make_key(score, idx0 + static_cast<uint32_t>(c)), node, a.n, lane,
-                     sinks);
-        }
-      }
-      if (pass == 1) zthr = zthreshold(wb.thr, s, lse);
-    }
-    if (pass == 0) {
-      __syncwarp();
-      refresh_thr(wb, ctl, a.n, C, lane, sinks);
-      zthr = zthreshold(wb.thr, s, lse);
-    }
-  }
+  m = warp_max(m);
+  if (t.lane == 0 && m > __int_as_float(0xFF800000)) atomicMax(&ctl->ref_ord[slot], ord_f32(m));
+  team_sync(t);
+  const unsigned o = *reinterpret_cast<volatile unsigned*>(&ctl->ref_ord[slot]);
+  if (t.tid == 0) ctl->ref_ord[slot ^ 1] = 0u;
+  return o ? unord_f32(o) : 0.f;
 }
 
+// --------------------------------------------------------------- kernel
 template <int BF16, int REG>
-__global__ void __launch_bounds__(REG ? kMaxStepThreadsReg : kMaxStepThreads, 1)
+__global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 32, 1)
     beam_step_kernel(const __grid_constant__ StepArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int kPerVec = BF16 ? 8 : 4;
   const StepConfig& cfg = a.cfg;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + cfg.off_bars);
-  uint64_t* empty = full + cfg.S;
   SelCtl* ctl = reinterpret_cast<SelCtl*>(smem + cfg.off_ctl);
-  Meta* meta = reinterpret_cast<Meta*>(smem + cfg.off_meta);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + cfg.off_bars);
   uint32_t* cta_hist = reinterpret_cast<uint32_t*>(smem + cfg.off_chist);
   uint32_t* whist = reinterpret_cast<uint32_t*>(smem + cfg.off_whist);
   uint32_t* wprefix = reinterpret_cast<uint32_t*>(smem + cfg.off_wprefix);
@@ -811,106 +749,240 @@ __global__ void __launch_bounds__(REG ? kMaxStepThreadsReg : kMaxStepThreads, 1)
   uint64_t* wkeys = reinterpret_cast<uint64_t*>(smem + cfg.off_wkeys);
   int32_t* wvals = reinterpret_cast<int32_t*>(smem + cfg.off_wvals);
 
+  const int W = cfg.W, S = cfg.S;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < cfg.S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], a.coop ? cfg.W : 1);
-      meta[s].seq = 0xFFFFFFFFu;
+  const Team team{static_cast<int>(threadIdx.x), W * 32, warp, lane, W};
+
+  int64_t lo, hi;
+  a.part.range(static_cast<int>(blockIdx.x), lo, hi);
+  RowSeq q;
+  if (a.coop) {
+    q = RowSeq{lo, 1, static_cast<int>(hi - lo)};
+  } else {
+    const int64_t f = lo + warp;
+    q = RowSeq{f, W, f < hi ? static_cast<int>((hi - f + W - 1) / W) : 0};
+  }
+  const int part = a.coop ? warp : 0;
+  const int nparts = a.coop ? W : 1;
+
+  Ring g{};
+  g.stages = stages + static_cast<size_t>(warp) * S * cfg.stage_bytes;
+  g.full = bars + warp * S;
+  g.S = S;
+  const uint64_t pol = policy_evict_first();
+
+  // 1. This warp's barriers, and the logits of its first S rows, before any
+  //    parent data is known (the rest of each stage follows below).
+  if (lane == 0) {
+    for (int k = 0; k < S; ++k) mbar_init(&g.full[k], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const int spec = q.count < S ? q.count : S;
+  if (lane == 0) {
+    for (int k = 0; k < spec; ++k) {
+      mbar_expect_tx(&g.full[k], static_cast<uint32_t>(cfg.logits_copy_bytes));
+      bulk_copy_g2s(g.stages + static_cast<size_t>(k) * cfg.stage_bytes,
+                    a.logits + q.row(k) * a.row_bytes,
+                    static_cast<uint32_t>(cfg.logits_copy_bytes), &g.full[k], pol);
     }
+  }
+  MetaBatch mb;
+  load_meta(a, q, 0, lane, mb);
+
+  // 2. CTA state, and the first segment's histogram reference.
+  if (threadIdx.x == 0) {
     ctl->cta_thr = 0ull;
     ctl->abort_flag = 0;
     ctl->counter = 0;
-    ctl->next_item = 0;
-    fence_mbar_init();
+    ctl->ref_ord[0] = 0u;
+    ctl->ref_ord[1] = 0u;
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
   __syncthreads();
+  const int r_first = static_cast<int>(lo / a.B_in);
+  const int r_last = static_cast<int>((hi - 1) / a.B_in);
+  int ref_slot = 0;
+  float C = segment_ref(a, team, ctl, r_first, ref_slot);
 
-  int64_t row_lo, row_hi;
-  a.part.range(static_cast<int>(blockIdx.x), row_lo, row_hi);
-
-  if (warp == 0) {
-    producer(a, stages, meta, full, empty, ctl, row_lo, row_hi, lane);
-    return;
+  // 3. Trie data of the first rows, now that their parents are known.
+  for (int k = 0; k < spec; ++k) {
+    const int live = (mb.live >> k) & 1u;
+    const float s = __shfl_sync(kFull, mb.s, k);
+    const int32_t p = __shfl_sync(kFull, mb.p, k);
+    const uint32_t o0 = __shfl_sync(kFull, mb.o0, k);
+    const uint32_t o1 = __shfl_sync(kFull, mb.o1, k);
+    if (lane == k) {
+      g.st_seq = k;
+      g.st_live = live;
+      g.st_s = s;
+      g.st_p = p;
+      g.st_o0 = o0;
+      g.st_o1 = o1;
+    }
+    if (lane == 0) {
+      const uint32_t ex = live ? extra_bytes(a, o0, o1) : 0u;
+      mbar_arrive_expect_tx(&g.full[k], ex);
+      if (ex) copy_extra(a, g.stages + static_cast<size_t>(k) * cfg.stage_bytes, &g.full[k], p, o0,
+                         ex, pol);
+    }
   }
+  g.issued = spec;
+  g.ip = spec;
 
-  Team team{static_cast<int>(threadIdx.x) - 32, cfg.W * 32, warp - 1, lane, cfg.W};
-  WarpBuf wb{wkeys + static_cast<size_t>(team.warp) * cfg.Cw,
-             wvals + static_cast<size_t>(team.warp) * cfg.Cw, whist + team.warp * 256, cfg.Cw,
-             0, 0ull, 0};
-  uint32_t* my_prefix = wprefix + team.warp * cfg.prefix_words;
-  uint32_t* my_mask = wmask + team.warp * cfg.prefix_words;
+  WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw,
+             wvals + static_cast<size_t>(warp) * cfg.Cw, whist + warp * 256, cfg.Cw, 0, 0ull, 0};
+  uint32_t* my_prefix = wprefix + warp * cfg.prefix_words;
+  uint32_t* my_mask = wmask + warp * cfg.prefix_words;
   const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
                           static_cast<uint32_t>(a.V)};
-  const int part = a.coop ? team.warp : 0;
-  const int nparts = a.coop ? cfg.W : 1;
+  const int direct_cap = (W * S * cfg.stage_bytes / 12) & ~1;
 
-  // Items are claimed in order from a shared counter (round-robin would let
-  // one slow row hold back the items queued behind it); in cooperative mode
-  // every warp takes every item.
-  uint32_t item = 0;
-  while (true) {
-    if (!a.coop) {
-      int claimed = 0;
-      if (lane == 0) claimed = atomicAdd(&ctl->next_item, 1);
-      item = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, claimed, 0));
+  // End of the segment of request cur_r (all warps, in the same order).
+  int cur_r = r_first;
+  auto flush = [&]() -> bool {
+    FlushArgs f;
+    f.n = a.n;
+    f.r = cur_r;
+    f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
+    f.G = a.part.contributors(cur_r);
+    f.maxG = a.part.maxG;
+    f.part_keys = a.part_keys;
+    f.part_vals = a.part_vals;
+    f.part_count = a.part_count;
+    f.tickets = a.tickets;
+    f.request_thr = a.request_thr;
+    f.ghist = a.ghist;
+    f.C = C;
+    f.wkeys = wkeys;
+    f.cw = cfg.Cw;
+    f.sort_keys = wkeys;
+    f.sort_vals = wvals;
+    f.sort_cap = W * cfg.Cw;
+    f.radix_hist = cta_hist;
+    f.wvals = wvals;
+    f.rank_P = whist;
+    f.rank_cur = whist + kHistBins;
+    // The stages are idle only at the CTA's last segment (every ring is empty).
+    const bool last = cur_r == r_last;
+    f.direct_keys = last ? reinterpret_cast<uint64_t*>(stages) : nullptr;
+    f.direct_vals = last ? reinterpret_cast<int32_t*>(stages + static_cast<size_t>(direct_cap) * 8)
+                         : nullptr;
+    f.direct_cap = last ? direct_cap : 0;
+    if (segment_flush(team, wb, ctl, f, writer)) return true;
+    if (cur_r < r_last) C = segment_ref(a, team, ctl, cur_r + 1, ref_slot ^= 1);
+    ++cur_r;
+    return false;
+  };
+
+  bool wait_failed = false, stopped = false;
+  unsigned long long req_pref = 0ull;
+  int req_pref_r = -1;
+  while (g.consumed < g.issued) {
+    const int stage = g.consumed % S;
+    if (!bounded_wait(&g.full[stage], (g.consumed / S) & 1u, &ctl->abort_flag, a.status,
+                      kStatusTimeout)) {
+      wait_failed = true;
+      break;
     }
-    const int stage = static_cast<int>(item % cfg.S);
-    const bool got = wait_item(meta, full, stage, item, static_cast<uint32_t>(cfg.S),
-                               &ctl->abort_flag, a.status);
-    Meta m;
-    int kind = kItemSegmentEnd;
-    if (got) {
-      m = meta[stage];
-      kind = m.kind;
-    } else {
-      m.req = -1;
+    const int seq = __shfl_sync(kFull, g.st_seq, stage);
+    const int live = __shfl_sync(kFull, g.st_live, stage);
+    const float s = __shfl_sync(kFull, g.st_s, stage);
+    const uint32_t o0 = __shfl_sync(kFull, g.st_o0, stage);
+    const uint32_t o1 = __shfl_sync(kFull, g.st_o1, stage);
+    const uint8_t* zrow = g.stages + static_cast<size_t>(stage) * cfg.stage_bytes;
+    if (!live) {
+      ++g.consumed;
+      ring_refill(a, q, mb, g, lane, pol);
+      continue;
     }
-    __syncwarp();
-    if (kind == kItemRow) {
-      const uint8_t* zrow = stages + static_cast<size_t>(stage) * cfg.stage_bytes;
-      const bool reg_ok = REG && (a.layout != SIDBEAM_LAYOUT_CSR ||
-                                  m.o1 - m.o0 <= static_cast<uint32_t>(32 * nparts));
-      if (reg_ok) {
-        process_row_reg<BF16>(a, zrow, &empty[stage], m, wb, ctl, my_mask, my_prefix, lane, part,
-                              nparts);
-      } else {
-        process_row_smem<BF16>(a, zrow, m, wb, ctl, my_prefix, lane, part, nparts);
+    const int64_t row = q.row(seq);
+    const int r = static_cast<int>(row) / a.B_in;  // rows number < 2^31
+    while (r > cur_r && !stopped) stopped = flush();
+    if (stopped) break;
+
+    const uint32_t b = static_cast<uint32_t>(row - static_cast<int64_t>(r) * a.B_in);
+    RowCtx c{s, 0.f, C, b * static_cast<uint32_t>(a.V), o0, o1};
+    const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
+    const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
+    req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+    req_pref_r = r;
+    const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
+    const bool reg_row = REG && (!csr || o1 - o0 <= static_cast<uint32_t>(32 * nparts));
+    if (reg_row) {
+      uint4 x[kRegVecs];
+      copy_row_regs<BF16>(zrow, a.V, lane, x);
+      if (a.layout == SIDBEAM_LAYOUT_DENSE) {  // mask_stride is a multiple of 4 words
+        const uint4* mrow = reinterpret_cast<const uint4*>(zrow + cfg.logits_copy_bytes);
+        for (int i = lane; i < (a.mask_stride >> 2); i += 32)
+          reinterpret_cast<uint4*>(my_mask)[i] = mrow[i];
+      }
+      const uint32_t ck = o0 + static_cast<uint32_t>(part * 32 + lane);
+      const bool cin = csr && ck < o1;
+      int ccode = 0;
+      float cz = 0.f;
+      if (cin) {
+        ccode = csr_code(a, zrow, o0, csr_staged(a, o0, o1), ck);
+        cz = elem<BF16>(zrow, ccode);
+      }
+      ++g.consumed;
+      ring_refill(a, q, mb, g, lane, pol);  // the stage is refilled before any arithmetic
+
+      const int nvec = (a.V + kPerVec - 1) / kPerVec;
+      float rmax;
+      row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
+      row_thresholds(wb, ctl, req_now);
+      float zthr = zthreshold(wb.thr, c.s, c.lse);
+      if (rmax < zthr) continue;
+      if (csr) {
+        bool ok = cin && cz >= zthr;
+        if (!__any_sync(kFull, ok)) continue;
+        const float score = c.s + (cz - c.lse);
+        warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
+        refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+        zthr = zthreshold(wb.thr, c.s, c.lse);
+        ok = cin && cz >= zthr;
+        warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(ccode)),
+                      static_cast<int32_t>(ck), static_cast<uint32_t>(a.n), lane, sinks);
+        continue;
       }
+      const uint32_t flags = vec_flags<BF16>(x, nvec, zthr, lane, part, nparts);
+      if (!__any_sync(kFull, flags != 0u)) continue;
+      bool have_prefix = false;
+      reg_extract<BF16, 0>(a, x, flags, my_mask, my_prefix, have_prefix, c, zthr, wb, ctl, sinks,
+                           lane);
+      __syncwarp();
+      refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+      zthr = zthreshold(wb.thr, c.s, c.lse);
+      reg_extract<BF16, 1>(a, x, flags, my_mask, my_prefix, have_prefix, c, zthr, wb, ctl, sinks,
+                           lane);
     } else {
-      if (got && lane == 0) mbar_arrive(&empty[stage]);
-      if (kind == kItemExit) {
-        team_sync_or(team, false);  // pairs with any warp that stops on an abort
-        break;
-      }
-      const int r = m.req;
-      FlushArgs f;
-      f.n = a.n;
-      f.r = r < 0 ? 0 : r;
-      f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(f.r);
-      f.G = a.part.contributors(f.r);
-      f.maxG = a.part.maxG;
-      f.part_keys = a.part_keys;
-      f.part_vals = a.part_vals;
-      f.part_count = a.part_count;
-      f.tickets = a.tickets;
-      f.request_thr = a.request_thr;
-      f.ghist = a.ghist;
-      f.C = m.C;
-      f.wkeys = wkeys;
-      f.cw = cfg.Cw;
-      f.sort_keys = wkeys;
-      f.sort_vals = wvals;
-      f.sort_cap = cfg.W * cfg.Cw;
-      f.radix_hist = cta_hist;
-      if (segment_flush(team, wb, ctl, f, writer)) break;
+      float rmax;
+      row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
+      row_thresholds(wb, ctl, req_now);
+      smem_walks<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
+                       sinks, lane, part, nparts);
+      __syncwarp();
+      ++g.consumed;
+      ring_refill(a, q, mb, g, lane, pol);
     }
-    if (a.coop) ++item;
   }
+
+  // 4. Remaining segment ends. A warp whose wait gave up has set the abort
+  //    flag; the next flush sees it in every warp and all of them stop.
+  if (!stopped) {
+    if (wait_failed) {
+      flush();
+    } else {
+      while (cur_r <= r_last)
+        if (flush()) break;
+    }
+  }
+  // Copies still in flight land before the CTA's shared memory goes away.
+  if (lane == 0)
+    for (int k = g.consumed; k < g.issued; ++k) drain_wait(&g.full[k % S], (k / S) & 1u);
 }
 
 }  // namespace
@@ -919,9 +991,11 @@ __global__ void __launch_bounds__(REG ? kMaxStepThreadsReg : kMaxStepThreads, 1)
 
 static int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Shared-memory plan: stage = logits row (16-byte rounded) + trie extra
-// (dense mask row / staged CSR codes); per consumer warp: top-n buffer,
-// radix histogram, dense prefix counts (and, on the register path, a mask copy).
+// Shared-memory plan: [control | barriers | radix scratch | warp histograms
+// (>= 2 x 1024 words: the rank merge's scratch) | dense prefix counts | mask
+// copies | W x S stages | W top-n buffers]. The first warp count (from 8 down)
+// that fits with at least two stages per warp wins; one stage per warp is the
+// last resort. Small rows get more stages (up to kMaxStages).
 bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int n, bool reg,
                         StepConfig* cfg) {
   StepConfig c{};
@@ -933,48 +1007,42 @@ bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int
   int npow2 = 1;
   while (npow2 < n) npow2 <<= 1;
   const int ctl_bytes = round_up(static_cast<int>(sizeof(dev::SelCtl)), 128);
-  const int meta_bytes = kMaxStages * static_cast<int>(sizeof(Meta));
-  static const int kWarpsSmem[] = {12, 10, 8, 6, 4, 3, 2, 1};
-  static const int kWarpsReg[] = {8, 6, 4, 3, 2, 1};
-  const int* warps = reg ? kWarpsReg : kWarpsSmem;
-  const int nw = reg ? 6 : 8;
-  for (int wi = 0; wi < nw; ++wi) {
-    const int W = warps[wi];
-    const int cw = std::max(round_up(n, 32) + 128, round_up((npow2 + W - 1) / W, 32));
-    int o = 0;
-    c.off_bars = o;
-    o += 2 * kMaxStages * 8;
-    c.off_ctl = o;
-    o += ctl_bytes;
-    c.off_meta = o;
-    o += meta_bytes;
-    c.off_chist = o;
-    o += 1024;
-    c.off_whist = o;
-    o += W * 1024;
-    c.off_wprefix = o;
-    o += W * c.prefix_words * 4;
-    c.off_wmask = o;
-    o += reg ? W * c.prefix_words * 4 : 0;
-    o = round_up(o, 128);
-    const int warp_bytes = W * cw * 12 + 256;
-    const int avail = kSmemBudget - o - warp_bytes;
-    if (avail < c.stage_bytes) continue;
-    const int S = std::min(kMaxStages, avail / c.stage_bytes);
-    if (S < 6 && W > 2) continue;
-    c.W = W;
-    c.S = S;
-    c.Cw = cw;
-    c.off_stage = o;
-    o += S * c.stage_bytes;
-    c.off_wkeys = round_up(o, 128);
-    o = c.off_wkeys + W * cw * 8;
-    c.off_wvals = round_up(o, 16);
-    o = c.off_wvals + W * cw * 4;
-    c.smem_bytes = round_up(o, 128);
-    if (c.smem_bytes > kSmemBudget) continue;
-    *cfg = c;
-    return true;
+  static const int kWarps[] = {8, 6, 4, 2, 1};
+  for (int min_s = 2; min_s >= 1; --min_s) {
+    for (int W : kWarps) {
+      const int cw = std::max(round_up(n, 32) + 128, round_up((npow2 + W - 1) / W, 32));
+      int o = 0;
+      c.off_ctl = o;
+      o += ctl_bytes;
+      c.off_bars = o;
+      o += round_up(W * kMaxStages * 8, 128);
+      c.off_chist = o;
+      o += 1024;
+      c.off_whist = o;
+      o += std::max(W * 1024, 2 * dev::kHistBins * 4);
+      c.off_wprefix = o;
+      o += W * c.prefix_words * 4;
+      c.off_wmask = o;
+      o += reg ? W * c.prefix_words * 4 : 0;
+      o = round_up(o, 128);
+      const int warp_bytes = W * cw * 12 + 256;
+      const int avail = kSmemBudget - o - warp_bytes;
+      const int S = std::min(kMaxStages, avail / (W * c.stage_bytes));
+      if (S < min_s) continue;
+      c.W = W;
+      c.S = S;
+      c.Cw = cw;
+      c.off_stage = o;
+      o += W * S * c.stage_bytes;
+      c.off_wkeys = round_up(o, 128);
+      o = c.off_wkeys + W * cw * 8;
+      c.off_wvals = round_up(o, 16);
+      o = c.off_wvals + W * cw * 4;
+      c.smem_bytes = round_up(o, 128);
+      if (c.smem_bytes > kSmemBudget) continue;
+      *cfg = c;
+      return true;
+    }
   }
   return false;
 }
@@ -1050,8 +1118,9 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
       !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, &a.cfg)))
     return set_error(SIDBEAM_ERR_INVALID_ARG,
                      "beam_step: V=%d with n_out=%d does not fit in shared memory", V, n_out);
+  if (a.cfg.W > (a.cfg.reg ? kMaxStepWarpsReg : kMaxStepWarps))
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: internal warp plan out of range");
   a.coop = a.part.rows_per_cta < a.cfg.W ? 1 : 0;
-  a.markers = a.coop ? 1 : a.cfg.W;
 
   const void* fns[4] = {reinterpret_cast<const void*>(&beam_step_kernel<0, 0>),
                         reinterpret_cast<const void*>(&beam_step_kernel<1, 0>),
@@ -1061,7 +1130,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   cudaError_t e = opt_in_smem(fns[which], which);
   if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaFuncSetAttribute");
   const dim3 grid(static_cast<unsigned>(a.part.grid));
-  const dim3 block(static_cast<unsigned>(32 * (a.cfg.W + 1)));
+  const dim3 block(static_cast<unsigned>(32 * a.cfg.W));
   switch (which) {
     case 0: beam_step_kernel<0, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 1: beam_step_kernel<1, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;

@@ -144,6 +144,12 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     f.ghist = a.ghist;
     f.C = C;
     f.radix_hist = cta_hist;
+    f.wvals = wvals;
+    f.rank_P = whist;  // the warps' radix scratch is free during a flush: 2 x 1024 words
+    f.rank_cur = whist + kHistBins;
+    f.direct_keys = nullptr;
+    f.direct_vals = nullptr;
+    f.direct_cap = 0;
     if (segment_flush(team, wb, ctl, f, writer)) return;
     seg_lo = seg_hi;
   }
@@ -154,6 +160,7 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 bool choose_score_config(int depth, int Vmax, int K, ScoreConfig* out) {
   ScoreConfig c{};
   c.W = kScoreWarps;
+  static_assert(kScoreWarps * 256 >= 2 * dev::kHistBins, "rank-merge scratch lives in whist");
   int npow2 = 1;
   while (npow2 < K) npow2 <<= 1;
   c.Cw = std::max(round_up(K, 32) + 512, round_up((npow2 + c.W - 1) / c.W, 32));

@@ -9,10 +9,10 @@
 
 namespace sidbeam {
 
-constexpr int kMaxStepThreads = 416;         // 1 producer + up to 12 consumer warps
-constexpr int kMaxStepThreadsReg = 288;      // register-row path: 1 producer + up to 8
-constexpr int kSmemBudget = 232448;          // 227 KiB of dynamic shared memory per CTA
-constexpr int kMaxStages = 32;
+constexpr int kMaxStepWarpsReg = 8;    // register-row kernel: up to 8 warps (<= 255 registers)
+constexpr int kMaxStepWarps = 12;      // shared-memory-row kernel
+constexpr int kSmemBudget = 232448;    // 227 KiB of dynamic shared memory per CTA
+constexpr int kMaxStages = 8;          // ring stages per warp
 
 // Rows [0, total_rows) in request-major order (row = r * B_in + b) are split
 // over CTAs. When there are at least as many CTAs as requests, each request
@@ -115,18 +115,19 @@ inline WorkspaceLayout workspace_layout(int R, int maxG, int n) {
   return w;
 }
 
-// Shared-memory plan of one beam_step CTA.
+// Shared-memory plan of one beam_step CTA: every warp owns a ring of S
+// stages (logits row + trie extra) that it fills itself with bulk copies.
 struct StepConfig {
-  int W;                  // consumer warps
-  int S;                  // ring stages
-  int Cw;                 // candidate slots per consumer warp (>= n + 32)
+  int W;                  // warps
+  int S;                  // ring stages per warp
+  int Cw;                 // candidate slots per warp (>= n + 32)
   int stage_bytes;
   int logits_copy_bytes;  // V * sizeof(dtype) rounded up to 16
   int extra_bytes;        // per stage after the row: dense mask row or staged CSR codes
-  int prefix_words;       // dense levels: per-warp set-bit prefix counts of a mask row
+  int prefix_words;       // dense levels: mask words per warp (prefix counts, mask copy)
   int reg;                // rows held in registers (<= 8 KB per row)
-  int off_bars, off_ctl, off_meta, off_chist, off_whist, off_wprefix, off_wmask, off_stage,
-      off_wkeys, off_wvals;
+  int off_ctl, off_bars, off_chist, off_whist, off_wprefix, off_wmask, off_stage, off_wkeys,
+      off_wvals;
   int smem_bytes;
 };
 

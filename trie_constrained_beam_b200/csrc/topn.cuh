@@ -27,10 +27,19 @@
 //     cut to the CTA's n best and written to the CTA's slot of the request's
 //     partial lists in global memory;
 //  3. request: the CTA that takes the last ticket (threadfence + atomic
-//     counter; nothing ever spins) reads the complete histogram, copies the
-//     partial entries above its bound into shared memory, selects the n best,
-//     sorts them (bitonic, descending), writes them out and zeroes the ticket,
-//     bound and histogram for the next call.
+//     counter; nothing ever spins) reads the complete histogram and ranks the
+//     partial entries (below), writes them out and zeroes the ticket, bound
+//     and histogram for the next call. A CTA that holds a whole request ranks
+//     its warp buffers directly, with no partial lists and no ticket.
+// Ranking by histogram: every candidate that reaches the top n was counted
+// exactly once, in the bin of its own fp32 score, so P[b] (the count in the
+// bins above b) is exactly the number of top-n members that outrank every
+// member of bin b. An entry's rank is P[b] plus the number of entries of its
+// own bin with a larger key; grouping the entries by bin (counting-sort
+// scatter) makes that a handful of compares per entry. Entries ranked >= n
+// are dropped. When a bin is too crowded (ties, a reference far off) or the
+// staging area too small, the entries are selected (radix walk) and sorted
+// (bitonic) instead.
 #pragma once
 
 #include "device_utils.cuh"
@@ -238,7 +247,8 @@ struct SelCtl {
   int is_last;
   int abort_flag;
   int staged;
-  int next_item;               // dynamic ring-item claims (beam_step)
+  int rank_bad;                // rank merge: the entries did not match the histogram
+  unsigned ref_ord[2];         // beam_step: max parent score (ordered) of a segment, by parity
   int wcount[32];
   int segoff[kMaxSegCounts + 1];
   __align__(16) uint32_t hist[kHistBins];  // score histogram of the current segment
@@ -395,6 +405,125 @@ __device__ inline void cta_bitonic_desc(const Team& t, uint64_t* keys, int32_t* 
   }
 }
 
+// ------------------------------------------------------------ rank merge
+// Entries with values: nseg lists (list s holds count(s) entries).
+struct WarpListSrc {  // warp buffers in shared memory, stride cw
+  const uint64_t* keys;
+  const int32_t* vals;
+  int cw;
+  const int* counts;
+  int nseg;
+  __device__ __forceinline__ int count(int s) const { return counts[s]; }
+  __device__ __forceinline__ uint64_t key(int s, int i) const { return keys[s * cw + i]; }
+  __device__ __forceinline__ int32_t val(int s, int i) const { return vals[s * cw + i]; }
+};
+struct PartialListSrc {  // one request's partial lists in global memory, stride n
+  const unsigned long long* keys;
+  const int32_t* vals;
+  int n;
+  const int* segoff;  // shared: list s holds segoff[s+1] - segoff[s] entries
+  int nseg;
+  __device__ __forceinline__ int count(int s) const { return segoff[s + 1] - segoff[s]; }
+  __device__ __forceinline__ uint64_t key(int s, int i) const {
+    return __ldcg(keys + static_cast<size_t>(s) * n + i);
+  }
+  __device__ __forceinline__ int32_t val(int s, int i) const {
+    return __ldcg(vals + static_cast<size_t>(s) * n + i);
+  }
+};
+
+// Compare budget of the in-bin ranking (sum over bins of count^2).
+constexpr uint32_t kRankWorkLimit = 1u << 18;
+
+// Ranks the entries of `src` by the complete score histogram `hist` (see the
+// header) and hands ranks 0..n-1 to `out`. Returns false, having written
+// nothing, when the entries must be selected and sorted instead (a crowded
+// bin, too little staging room, or entries that do not match the histogram).
+// P and cur: 1024 words of shared scratch each; stk/stv: `cap` staging slots.
+// All team threads call it; the result is the same for all of them.
+template <class Src, class Writer>
+__device__ bool rank_merge(const Team& t, SelCtl* ctl, const uint32_t* hist, const Src& src,
+                           uint32_t n, int r, float C, uint64_t* stk, int32_t* stv, int cap,
+                           uint32_t* P, uint32_t* cur, const Writer& out) {
+  // 1. Exclusive prefix counts, the bin bK of the n-th best and the work.
+  if (t.warp == 0) {
+    uint32_t carry = 0, work = 0;
+    int bK = -1;
+    for (int i = 0; i < kHistBins / 32; ++i) {
+      const int b = 32 * i + t.lane;
+      const uint32_t c = hist[b];
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (t.lane >= o) incl += y;
+      }
+      const uint32_t excl = carry + incl - c;
+      P[b] = excl;
+      cur[b] = 0u;
+      if (bK < 0) {
+        const unsigned hit = __ballot_sync(0xFFFFFFFFu, excl + c >= n);
+        if (hit) bK = 32 * i + __ffs(hit) - 1;
+        const uint32_t cc = c < 4096u ? c : 4096u;
+        const uint32_t sq = (bK < 0 || b <= bK) ? cc * cc : 0u;
+        work += warp_sum_u(sq);
+      }
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    if (bK < 0) bK = kHistBins - 1;  // fewer than n candidates: all of them rank
+    if (t.lane == 0) {
+      const uint32_t total = P[bK] + hist[bK];
+      ctl->bcast_d = bK;
+      ctl->bcast_cnt = total;
+      ctl->bcast_above = (total <= static_cast<uint32_t>(cap) && work <= kRankWorkLimit) ? 1u : 0u;
+      ctl->rank_bad = 0;
+    }
+  }
+  team_sync(t);
+  if (!ctl->bcast_above) return false;
+  const int bK = ctl->bcast_d;
+  const int total = static_cast<int>(ctl->bcast_cnt);
+  for (int i = t.tid; i < total; i += t.T) stk[i] = 0ull;
+  team_sync(t);
+  // 2. Scatter the entries of bins 0..bK into their bins' slot ranges.
+  for (int s = 0; s < src.nseg; ++s) {
+    const int c = src.count(s);
+    for (int i = t.tid; i < c; i += t.T) {
+      const uint64_t key = src.key(s, i);
+      if (key == 0ull) continue;
+      const uint32_t b = score_bin(key_score(key), C);
+      if (b > static_cast<uint32_t>(bK)) continue;
+      const uint32_t slot = P[b] + atomicAdd(&cur[b], 1u);
+      if (slot < P[b] + hist[b]) {
+        stk[slot] = key;
+        stv[slot] = src.val(s, i);
+      } else {
+        ctl->rank_bad = 1;
+      }
+    }
+  }
+  team_sync(t);
+  // Every bin above bK must be complete (all its candidates rank < n).
+  for (int b = t.tid; b < bK; b += t.T)
+    if (cur[b] != hist[b]) ctl->rank_bad = 1;
+  team_sync(t);
+  if (ctl->rank_bad) return false;
+  // 3. Rank = entries in the bins above + larger keys of the same bin.
+  const int filled = static_cast<int>(P[bK] + cur[bK]);
+  for (int i = t.tid; i < filled; i += t.T) {
+    const uint64_t key = stk[i];
+    const uint32_t b = score_bin(key_score(key), C);
+    const uint32_t lo = P[b], hi = lo + cur[b];
+    uint32_t rank = lo;
+    for (uint32_t j = lo; j < hi; ++j) rank += stk[j] > key ? 1u : 0u;
+    if (rank < n) out(r, static_cast<int>(rank), key, stv[i], true);
+  }
+  for (int i = (filled < static_cast<int>(n) ? filled : static_cast<int>(n)) + t.tid;
+       i < static_cast<int>(n); i += t.T)
+    out(r, i, 0ull, -1, false);
+  return true;
+}
+
 // ------------------------------------------------------------ warp buffers
 struct WarpBuf {
   uint64_t* keys;   // [cw] shared
@@ -448,6 +577,45 @@ __device__ __forceinline__ void warp_compact(WarpBuf& wb, uint32_t n, int lane,
   if (K > wb.thr) wb.thr = K;
   publish_thr(K, lane, sinks);
   __syncwarp();
+}
+
+// warp_compact behind a call (for code that offers from many unrolled sites:
+// the rare compaction then exists once instead of once per site).
+struct CompactOut {
+  uint64_t thr;
+  int count;
+};
+static __device__ __noinline__ CompactOut warp_compact_call(uint64_t* keys, int32_t* vals, uint32_t* hist,
+                                                     int cw, int count, uint64_t thr, uint32_t n,
+                                                     int lane, unsigned long long* cta_thr,
+                                                     unsigned long long* request_thr) {
+  WarpBuf wb{keys, vals, hist, cw, count, thr, 0};
+  warp_compact(wb, n, lane, ThrSinks{cta_thr, request_thr});
+  return CompactOut{wb.thr, wb.count};
+}
+
+// warp_offer with the compaction behind a call.
+__device__ __forceinline__ void warp_offer_nc(WarpBuf& wb, bool valid, uint64_t key, int32_t val,
+                                              uint32_t n, int lane, const ThrSinks& sinks) {
+  bool pass = valid && key >= wb.thr;
+  unsigned bal = __ballot_sync(0xFFFFFFFFu, pass);
+  if (bal == 0) return;
+  int cnt = __popc(bal);
+  if (wb.count + cnt > wb.cw) {
+    const CompactOut c = warp_compact_call(wb.keys, wb.vals, wb.hist, wb.cw, wb.count, wb.thr, n,
+                                           lane, sinks.cta_thr, sinks.request_thr);
+    wb.count = c.count;
+    wb.thr = c.thr;
+    pass = pass && key >= wb.thr;
+    bal = __ballot_sync(0xFFFFFFFFu, pass);
+    cnt = __popc(bal);
+  }
+  if (pass) {
+    const int pos = wb.count + __popc(bal & lanemask_lt());
+    wb.keys[pos] = key;
+    wb.vals[pos] = val;
+  }
+  wb.count += cnt;
 }
 
 // Offer one candidate per lane (only lanes with valid = true). Warp-collective:
@@ -515,6 +683,12 @@ struct FlushArgs {
   int32_t* sort_vals;
   int sort_cap;           // entries available at sort_keys / sort_vals
   uint32_t* radix_hist;   // 256-word scratch for cta_select
+  int32_t* wvals;         // all warp buffers' values, [nwarps][cw]
+  uint32_t* rank_P;       // 1024-word scratch for the rank merge (null: no rank merge)
+  uint32_t* rank_cur;     // 1024-word scratch for the rank merge
+  uint64_t* direct_keys;  // staging for ranking a whole request held by this CTA
+  int32_t* direct_vals;   //   (null when no free area is available)
+  int direct_cap;
 };
 
 // Warp-aggregated append position: this lane's slot among the `keep` lanes.
@@ -574,6 +748,17 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
   const int total = ctl->segoff[G];
   const unsigned long long* lists = f.part_keys + list0 * f.n;
   const int32_t* lvals = f.part_vals + list0 * f.n;
+  if (f.rank_P &&
+      rank_merge(t, ctl, ctl->hist, PartialListSrc{lists, lvals, f.n, ctl->segoff, G},
+                 static_cast<uint32_t>(f.n), f.r, f.C, f.sort_keys, f.sort_vals, f.sort_cap,
+                 f.rank_P, f.rank_cur, out)) {
+    for (int i = t.tid; i < kHistBins; i += t.T) gh[i] = 0u;
+    if (t.tid == 0) {
+      f.tickets[f.r] = 0u;
+      f.request_thr[f.r] = 0ull;
+    }
+    return;
+  }
   // Filtered copy of all partial entries >= K0 into [0, cap): flat index,
   // segment found by binary search, four independent loads per thread.
   uint64_t* stk = f.sort_keys;
@@ -744,6 +929,21 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
                               const Writer& out) {
   if (t.lane == 0) ctl->wcount[t.warp] = wb.count;
   if (team_sync_or(t, ctl->abort_flag != 0)) return true;
+  if (f.G == 1 && f.direct_keys && f.rank_P &&
+      rank_merge(t, ctl, ctl->hist, WarpListSrc{f.wkeys, f.wvals, f.cw, ctl->wcount, t.nwarps},
+                 static_cast<uint32_t>(f.n), f.r, f.C, f.direct_keys, f.direct_vals,
+                 f.direct_cap, f.rank_P, f.rank_cur, out)) {
+    team_sync(t);
+    for (int i = t.tid; i < kHistBins; i += t.T) ctl->hist[i] = 0u;
+    wb.count = 0;
+    wb.thr = 0;
+    if (t.tid == 0) {
+      ctl->cta_thr = 0ull;
+      f.request_thr[f.r] = 0ull;
+    }
+    team_sync(t);
+    return false;
+  }
   // 1. Add this segment's histogram to the request's (read back only by the
   //    merging CTA); bound the flush by this CTA's histogram and the shared bounds.
   uint32_t* gh = f.ghist + static_cast<size_t>(f.r) * kHistBins;
