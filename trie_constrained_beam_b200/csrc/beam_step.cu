@@ -45,6 +45,9 @@ using namespace dev;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRegVecs = 16;  // 16-byte vectors per lane held in registers (8 KB rows)
+// Dense rows with more children than this (per warp taking part) are walked in
+// place in their stage, in two passes, instead of from registers.
+constexpr uint32_t kHeavyDense = 128;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // f(I) for I = 0 .. N-1 with I a compile-time constant (keeps register arrays
@@ -273,7 +276,9 @@ __device__ __forceinline__ void vec_cut(uint4& x, int keep) {
 
 // Row max and log-normaliser of a row held in registers (vector lane + 32k in
 // x[k]; entries past V are -inf and contribute exp(-inf) = 0).
-template <int BF16>
+// FULL: every lane holds kRegVecs real vectors (a full 8 KB row); the loops
+// are then straight-line code the compiler can interleave freely.
+template <int BF16, bool FULL = false>
 __device__ __forceinline__ void row_stats_reg(const uint4 (&x)[kRegVecs], int nvec, int lane,
                                               float& m_out, float& lse_out) {
   float m;
@@ -281,14 +286,14 @@ __device__ __forceinline__ void row_stats_reg(const uint4 (&x)[kRegVecs], int nv
     uint32_t r = 0xFF80FF80u;
     Unrolled<kRegVecs>::run([&](auto kc) {
       constexpr int k = decltype(kc)::value;
-      if (32 * k < nvec) r = bmax2(r, bmax2(bmax2(x[k].x, x[k].y), bmax2(x[k].z, x[k].w)));
+      if (FULL || 32 * k < nvec) r = bmax2(r, bmax2(bmax2(x[k].x, x[k].y), bmax2(x[k].z, x[k].w)));
     });
     m = fmaxf(bf_lo(r), bf_hi(r));
   } else {
     m = __int_as_float(0xFF800000);
     Unrolled<kRegVecs>::run([&](auto kc) {
       constexpr int k = decltype(kc)::value;
-      if (32 * k < nvec) m = fmaxf(m, vec_max<0>(x[k]));
+      if (FULL || 32 * k < nvec) m = fmaxf(m, vec_max<0>(x[k]));
     });
   }
   // Lane-local max for the exponentials; lanes combined once at the end.
@@ -298,7 +303,7 @@ __device__ __forceinline__ void row_stats_reg(const uint4 (&x)[kRegVecs], int nv
   uint64_t a0 = 0, a1 = 0;
   Unrolled<kRegVecs>::run([&](auto kc) {
     constexpr int k = decltype(kc)::value;
-    if (32 * k < nvec) {
+    if (FULL || 32 * k < nvec) {
       if (k & 1) a1 = fadd2(a1, vec_sumexp2<BF16>(x[k], l2e, nml));
       else a0 = fadd2(a0, vec_sumexp2<BF16>(x[k], l2e, nml));
     }
@@ -536,133 +541,122 @@ __device__ __forceinline__ void copy_row_regs(const uint8_t* zrow, int V, int la
   });
 }
 
-// x[k] for a warp-uniform runtime k, through constant indices only (a
-// register array indexed at run time would be moved to local memory).
-__device__ __forceinline__ uint4 pick_vec(const uint4 (&x)[kRegVecs], int k) {
-  switch (k) {
-    case 0: return x[0];
-    case 1: return x[1];
-    case 2: return x[2];
-    case 3: return x[3];
-    case 4: return x[4];
-    case 5: return x[5];
-    case 6: return x[6];
-    case 7: return x[7];
-    case 8: return x[8];
-    case 9: return x[9];
-    case 10: return x[10];
-    case 11: return x[11];
-    case 12: return x[12];
-    case 13: return x[13];
-    case 14: return x[14];
-    default: return x[15];
-  }
-}
-
-// Bit k set: this lane's vector k (lane + 32k) is this warp's to walk and its
-// largest logit reaches the threshold.
-template <int BF16>
-__device__ __forceinline__ uint32_t vec_flags(const uint4 (&x)[kRegVecs], int nvec, float zthr,
-                                              int lane, int part, int nparts) {
-  uint32_t f = 0u;
-  Unrolled<kRegVecs>::run([&](auto kc) {
-    constexpr int k = decltype(kc)::value;
-    if (32 * k < nvec && (k % nparts) == part && lane + 32 * k < nvec &&
-        vec_max<BF16>(x[k]) >= zthr)
-      f |= 1u << k;
-  });
-  return f;
-}
-
-// One walk over the flagged vectors of a register row at a dense level or
-// without a trie. PASS 0 counts the children at or above the threshold in the
-// CTA histogram; PASS 1 offers them (re-testing each vector against the
-// raised threshold). The loop runs over vectors flagged in any lane.
-template <int BF16, int PASS>
-__device__ __forceinline__ void reg_extract(const StepArgs& a, const uint4 (&x)[kRegVecs],
-                                            uint32_t flags, const uint32_t* wmask,
-                                            uint32_t* wprefix, bool& have_prefix,
-                                            const RowCtx& c, float& zthr, WarpBuf& wb,
-                                            SelCtl* ctl, const ThrSinks& sinks, int lane) {
+// Children at or above the threshold in a register row (dense level or no
+// trie): byte k of the packed hits holds the bits of this lane's vector k
+// (lane + 32k) whose code is a valid child with z >= zthr. Only vectors whose
+// largest logit reaches the threshold look at the mask. Returns whether any
+// lane of the warp has a hit.
+template <int BF16, bool FULL>
+__device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRegVecs], int nvec,
+                                         float zthr, const uint32_t* wmask, int lane, int part,
+                                         int nparts, uint32_t (&hp)[kRegVecs / 4]) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  uint32_t todo = __reduce_or_sync(kFull, flags);
-  while (todo) {
-    const int k = __ffs(todo) - 1;
-    todo &= todo - 1u;
-    const uint4 xk = pick_vec(x, k);
+#pragma unroll
+  for (int i = 0; i < kRegVecs / 4; ++i) hp[i] = 0u;
+  Unrolled<kRegVecs>::run([&](auto kc) {
+    constexpr int k = decltype(kc)::value;
     const int v = lane + 32 * k;
-    unsigned bits = 0u;
-    if (((flags >> k) & 1u) && (PASS == 0 || vec_max<BF16>(xk) >= zthr)) {
+    const bool mine = FULL || (32 * k < nvec && (k % nparts) == part && v < nvec);
+    if (mine && vec_max<BF16>(x[k]) >= zthr) {
       const int cb = v * kPerVec;
       unsigned valid = (1u << kPerVec) - 1u;
       if (dense)
         valid = BF16 ? static_cast<unsigned>(reinterpret_cast<const uint8_t*>(wmask)[v])
                      : (wmask[v >> 3] >> ((v & 7) * 4)) & 0xFu;
-      if (a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+      if (!FULL && a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+      unsigned bits = 0u;
 #pragma unroll
       for (int j = 0; j < kPerVec; ++j)
-        if (((valid >> j) & 1u) && vec_elem<BF16>(xk, j) >= zthr) bits |= 1u << j;
+        if (((valid >> j) & 1u) && vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
+      hp[k >> 2] |= bits << ((k & 3) * 8);
     }
-    while (__any_sync(kFull, bits != 0u)) {
-      const bool has = bits != 0u;
-      const int j = has ? __ffs(bits) - 1 : 0;
-      bits &= bits - 1u;
-      const int code = v * kPerVec + j;
-      const float score = c.s + (vec_elem<BF16>(xk, j) - c.lse);
-      if (PASS == 0) {
-        warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned);
-      } else {
-        if (dense && !have_prefix) {
-          dense_prefix(wmask, a.mask_words, wprefix, lane);
-          have_prefix = true;
-        }
-        const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code) : -1;
-        warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
-                      static_cast<uint32_t>(a.n), lane, sinks);
+  });
+  return __any_sync(kFull, (hp[0] | hp[1] | hp[2] | hp[3]) != 0u);
+}
+
+// Counts every hit in the CTA histogram and offers it to the warp buffer (one
+// pass; a hit that falls below a threshold raised meanwhile is dropped). The
+// logits of the hits are read again from the row in global memory (it was
+// just streamed, so from L2): four per lane per round trip, one compact loop
+// instead of a copy of the walk per register vector.
+template <int BF16>
+__device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* grow,
+                                          const uint32_t (&hp)[kRegVecs / 4],
+                                          const uint32_t* wmask, uint32_t* wprefix,
+                                          const RowCtx& c, float& zthr, WarpBuf& wb, SelCtl* ctl,
+                                          const ThrSinks& sinks, int lane) {
+  constexpr int kPerVec = BF16 ? 8 : 4;
+  constexpr int kBatch = 4;
+  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
+  if (dense) dense_prefix(wmask, a.mask_words, wprefix, lane);
+  uint32_t hb[kRegVecs / 4] = {hp[0], hp[1], hp[2], hp[3]};
+  while (__any_sync(kFull, (hb[0] | hb[1] | hb[2] | hb[3]) != 0u)) {
+    int code[kBatch];
+    float z[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      int bit = -1;
+#pragma unroll
+      for (int w = kRegVecs / 4 - 1; w >= 0; --w)  // lowest set bit over the 128
+        if (hb[w]) bit = 32 * w + __ffs(hb[w]) - 1;
+      if (bit >= 0) hb[bit >> 5] &= hb[bit >> 5] - 1u;
+      code[u] = bit < 0 ? -1 : (lane + 32 * (bit >> 3)) * kPerVec + (bit & 7);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      z[u] = 0.f;
+      if (code[u] >= 0) {
+        if (BF16)
+          z[u] = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(grow) + code[u])) << 16);
+        else
+          z[u] = __ldg(reinterpret_cast<const float*>(grow) + code[u]);
       }
     }
-    if (PASS == 1) zthr = zthreshold(wb.thr, c.s, c.lse);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const bool has = code[u] >= 0 && z[u] >= zthr;
+      if (!__any_sync(kFull, has)) continue;
+      const float score = c.s + (z[u] - c.lse);
+      warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
+      const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code[u]) : -1;
+      warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code[u])), node,
+                    static_cast<uint32_t>(a.n), lane, sinks);
+      zthr = zthreshold(wb.thr, c.s, c.lse);
+    }
   }
 }
 
-// Candidate walks of a row in place in its stage (rows over 8 KB, or CSR rows
-// with more children than one 32-lane batch per warp).
+// Candidate walk of a row in place in its stage (rows over 8 KB, CSR rows with
+// more children than one 32-lane batch per warp, dense rows with many
+// children).
 template <int BF16>
-__device__ void smem_walks(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
-                           float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
-                           const ThrSinks& sinks, int lane, int part, int nparts) {
+__device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
+                          float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
+                          const ThrSinks& sinks, int lane, int part, int nparts) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   if (rmax < zthr) return;  // even the row's largest logit cannot reach the threshold
   if (a.layout == SIDBEAM_LAYOUT_CSR) {
     const uint32_t nst = csr_staged(a, c.o0, c.o1);
     const uint32_t k_step = static_cast<uint32_t>(32 * nparts);
-    const uint32_t k_begin = c.o0 + static_cast<uint32_t>(part * 32);
-    for (int pass = 0; pass < 2; ++pass) {
-      for (uint32_t k0 = k_begin; k0 < c.o1; k0 += k_step) {
-        const uint32_t k = k0 + lane;
-        const bool in = k < c.o1;
-        const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
-        const float z = in ? elem<BF16>(zrow, code) : 0.f;
-        const bool ok = in && z >= zthr;
-        if (!__any_sync(kFull, ok)) continue;
-        const float score = c.s + (z - c.lse);
-        if (pass == 0) {
-          warp_bin(ctl->hist, ok, score_bin(score, c.C), wb.binned);
-        } else {
-          warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(code)),
-                        static_cast<int32_t>(k), static_cast<uint32_t>(a.n), lane, sinks);
-          zthr = zthreshold(wb.thr, c.s, c.lse);
-        }
-      }
-      if (pass == 0) {
-        __syncwarp();
-        refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), c.C, lane, sinks);
-        zthr = zthreshold(wb.thr, c.s, c.lse);
-      }
+    for (uint32_t k0 = c.o0 + static_cast<uint32_t>(part * 32); k0 < c.o1; k0 += k_step) {
+      const uint32_t k = k0 + lane;
+      const bool in = k < c.o1;
+      const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
+      const float z = in ? elem<BF16>(zrow, code) : 0.f;
+      const bool ok = in && z >= zthr;
+      if (!__any_sync(kFull, ok)) continue;
+      const float score = c.s + (z - c.lse);
+      warp_bin(ctl->hist, ok, score_bin(score, c.C), wb.binned, &ctl->hist_total);
+      warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(code)),
+                    static_cast<int32_t>(k), static_cast<uint32_t>(a.n), lane, sinks);
+      zthr = zthreshold(wb.thr, c.s, c.lse);
     }
     return;
   }
+  // Dense level or no trie: many children, so two passes: count every child
+  // at or above the threshold, raise the threshold from the histogram, then
+  // offer only what still reaches it.
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
   const uint32_t* mrow = reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes);
   const int nvec_all = (a.V + kPerVec - 1) / kPerVec;
@@ -689,20 +683,21 @@ __device__ void smem_walks(const StepArgs& a, const uint8_t* zrow, const RowCtx&
         have_prefix = true;
       }
       while (__any_sync(kFull, bits != 0u)) {
-        const bool has = bits != 0u;
-        const int j = has ? __ffs(bits) - 1 : 0;
-        bits &= bits - 1u;
+        const int j = bits ? __ffs(bits) - 1 : 0;
         const int code = v * kPerVec + j;
-        const float score = has ? c.s + (elem<BF16>(zrow, code) - c.lse) : 0.f;
+        const float z = bits ? elem<BF16>(zrow, code) : 0.f;
+        const bool has = bits != 0u && z >= zthr;
+        bits &= bits - 1u;
+        const float score = c.s + (z - c.lse);
         if (pass == 0) {
-          warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned);
+          warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
         } else {
           const int32_t node = (has && dense) ? dense_child(mrow, wprefix, c.o0, code) : -1;
           warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
                         static_cast<uint32_t>(a.n), lane, sinks);
+          zthr = zthreshold(wb.thr, c.s, c.lse);
         }
       }
-      if (pass == 1) zthr = zthreshold(wb.thr, c.s, c.lse);
     }
     if (pass == 0) {
       __syncwarp();
@@ -798,6 +793,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     ctl->counter = 0;
     ctl->ref_ord[0] = 0u;
     ctl->ref_ord[1] = 0u;
+    ctl->hist_total = 0u;
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
   __syncthreads();
@@ -848,6 +844,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
     f.G = a.part.contributors(cur_r);
     f.maxG = a.part.maxG;
+    f.pcap = partial_cap(a.n);
     f.part_keys = a.part_keys;
     f.part_vals = a.part_vals;
     f.part_count = a.part_count;
@@ -906,10 +903,11 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     RowCtx c{s, 0.f, C, b * static_cast<uint32_t>(a.V), o0, o1};
     const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
     const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
-    req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
-    req_pref_r = r;
     const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
-    const bool reg_row = REG && (!csr || o1 - o0 <= static_cast<uint32_t>(32 * nparts));
+    const uint32_t nchild = o1 - o0;
+    const bool reg_row =
+        REG && (csr ? nchild <= static_cast<uint32_t>(32 * nparts)
+                    : (a.layout != SIDBEAM_LAYOUT_DENSE || nchild <= kHeavyDense * nparts));
     if (reg_row) {
       uint4 x[kRegVecs];
       copy_row_regs<BF16>(zrow, a.V, lane, x);
@@ -928,45 +926,49 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
       }
       ++g.consumed;
       ring_refill(a, q, mb, g, lane, pol);  // the stage is refilled before any arithmetic
+      req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+      req_pref_r = r;
 
       const int nvec = (a.V + kPerVec - 1) / kPerVec;
+      const bool full = nvec == 32 * kRegVecs && a.V % kPerVec == 0;
       float rmax;
-      row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
+      if (full)
+        row_stats_reg<BF16, true>(x, nvec, lane, rmax, c.lse);
+      else
+        row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
       float zthr = zthreshold(wb.thr, c.s, c.lse);
       if (rmax < zthr) continue;
       if (csr) {
-        bool ok = cin && cz >= zthr;
+        const bool ok = cin && cz >= zthr;
         if (!__any_sync(kFull, ok)) continue;
         const float score = c.s + (cz - c.lse);
-        warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned);
-        __syncwarp();
-        refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
-        zthr = zthreshold(wb.thr, c.s, c.lse);
-        ok = cin && cz >= zthr;
+        warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned, &ctl->hist_total);
         warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(ccode)),
                       static_cast<int32_t>(ck), static_cast<uint32_t>(a.n), lane, sinks);
-        continue;
+      } else {
+        uint32_t hp[kRegVecs / 4];
+        const bool any = (full && nparts == 1)
+                             ? reg_hits<BF16, true>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp)
+                             : reg_hits<BF16, false>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
+        if (!any) continue;
+        take_hits<BF16>(a, a.logits + row * a.row_bytes, hp, my_mask, my_prefix, c, zthr, wb,
+                        ctl, sinks, lane);
       }
-      const uint32_t flags = vec_flags<BF16>(x, nvec, zthr, lane, part, nparts);
-      if (!__any_sync(kFull, flags != 0u)) continue;
-      bool have_prefix = false;
-      reg_extract<BF16, 0>(a, x, flags, my_mask, my_prefix, have_prefix, c, zthr, wb, ctl, sinks,
-                           lane);
       __syncwarp();
       refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
-      zthr = zthreshold(wb.thr, c.s, c.lse);
-      reg_extract<BF16, 1>(a, x, flags, my_mask, my_prefix, have_prefix, c, zthr, wb, ctl, sinks,
-                           lane);
     } else {
       float rmax;
       row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
-      smem_walks<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
-                       sinks, lane, part, nparts);
+      smem_walk<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
+                      sinks, lane, part, nparts);
       __syncwarp();
+      refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
       ++g.consumed;
       ring_refill(a, q, mb, g, lane, pol);
+      req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+      req_pref_r = r;
     }
   }
 
@@ -1007,10 +1009,19 @@ bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int
   int npow2 = 1;
   while (npow2 < n) npow2 <<= 1;
   const int ctl_bytes = round_up(static_cast<int>(sizeof(dev::SelCtl)), 128);
-  static const int kWarps[] = {8, 6, 4, 2, 1};
-  for (int min_s = 2; min_s >= 1; --min_s) {
-    for (int W : kWarps) {
-      const int cw = std::max(round_up(n, 32) + 128, round_up((npow2 + W - 1) / W, 32));
+  // Register rows: 12 warps with one stage each (more warps hide more
+  // latency; the stage is refilled as soon as the row is in registers).
+  // Rows worked on in place: at least two stages per warp.
+  struct Plan { int W, min_s; };
+  static const Plan kRegPlans[] = {{12, 1}, {8, 2}, {8, 1}, {6, 1}, {4, 1}, {2, 1}, {1, 1}};
+  static const Plan kSmemPlans[] = {{8, 2}, {6, 2}, {4, 2}, {8, 1}, {6, 1}, {4, 1}, {2, 1}, {1, 1}};
+  const Plan* plans = reg ? kRegPlans : kSmemPlans;
+  const int nplans = reg ? 7 : 8;
+  for (int pi = 0; pi < nplans; ++pi) {
+    {
+      const int W = plans[pi].W, min_s = plans[pi].min_s;
+      if (W > (reg ? kMaxStepWarpsReg : kMaxStepWarps)) continue;
+      const int cw = std::max(round_up(n, 32) + 32, round_up((npow2 + W - 1) / W, 32));
       int o = 0;
       c.off_ctl = o;
       o += ctl_bytes;

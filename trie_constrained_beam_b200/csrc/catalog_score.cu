@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     ctl->cta_thr = 0ull;
     ctl->abort_flag = 0;
     ctl->counter = 0;
+    ctl->hist_total = 0u;
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
   WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw, wvals + static_cast<size_t>(warp) * cfg.Cw,
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
       const uint64_t key = make_key(score, static_cast<uint32_t>(j));
       const bool pass = valid && key >= wb.thr;
       if (!__any_sync(0xFFFFFFFFu, pass)) continue;
-      warp_bin(ctl->hist, pass, score_bin(score, C), wb.binned);
+      warp_bin(ctl->hist, pass, score_bin(score, C), wb.binned, &ctl->hist_total);
       if ((++batches & 7) == 0) refresh_thr(wb, ctl, static_cast<uint32_t>(a.K), C, lane, sinks);
       warp_offer(wb, pass, key, static_cast<int32_t>(j), static_cast<uint32_t>(a.K), lane, sinks);
     }
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(r);
     f.G = a.part.contributors(r);
     f.maxG = a.part.maxG;
+    f.pcap = partial_cap(a.K);
     f.part_keys = a.part_keys;
     f.part_vals = a.part_vals;
     f.part_count = a.part_count;

@@ -9,7 +9,7 @@
 
 namespace sidbeam {
 
-constexpr int kMaxStepWarpsReg = 8;    // register-row kernel: up to 8 warps (<= 255 registers)
+constexpr int kMaxStepWarpsReg = 12;   // register-row kernel: up to 12 warps (<= 168 registers)
 constexpr int kMaxStepWarps = 12;      // shared-memory-row kernel
 constexpr int kSmemBudget = 232448;    // 227 KiB of dynamic shared memory per CTA
 constexpr int kMaxStages = 8;          // ring stages per warp
@@ -86,7 +86,7 @@ inline Partition make_partition(int R, int64_t B_in, int ctas) {
 }
 
 // Workspace: [status | tickets[R] | request_thr[R] | score histograms[R][1024] |
-//             part_count[R][maxG] | part_keys[R][maxG][n] | part_vals[R][maxG][n]],
+//             part_count[R][maxG] | part_keys[R][maxG][2n] | part_vals[R][maxG][2n]],
 // 256-byte aligned parts. Everything before part_keys must start at zero.
 struct WorkspaceLayout {
   size_t status, tickets, request_thr, ghist, part_count, part_keys, part_vals, total;
@@ -94,7 +94,13 @@ struct WorkspaceLayout {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Entries a CTA may leave in its partial list of a request: 2n, so that the
+// survivors of a segment (the n best plus the slack of the histogram bound)
+// are written without an exact cut in the common case.
+__host__ __device__ __forceinline__ int partial_cap(int n) { return 2 * n; }
+
 inline WorkspaceLayout workspace_layout(int R, int maxG, int n) {
+  const int pcap = partial_cap(n);
   WorkspaceLayout w{};
   size_t o = 0;
   w.status = o;
@@ -108,9 +114,9 @@ inline WorkspaceLayout workspace_layout(int R, int maxG, int n) {
   w.part_count = o;
   o = align256(o + static_cast<size_t>(R) * maxG * 4);
   w.part_keys = o;
-  o = align256(o + static_cast<size_t>(R) * maxG * n * 8);
+  o = align256(o + static_cast<size_t>(R) * maxG * pcap * 8);
   w.part_vals = o;
-  o = align256(o + static_cast<size_t>(R) * maxG * n * 4);
+  o = align256(o + static_cast<size_t>(R) * maxG * pcap * 4);
   w.total = o;
   return w;
 }

@@ -133,9 +133,12 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, bool active, uint32_t b
 
 // Score-histogram increment by a whole warp; counts the additions for the
 // refresh policy. Warp-collective.
-__device__ __forceinline__ void warp_bin(uint32_t* hist, bool active, uint32_t bin, int& binned) {
+__device__ __forceinline__ void warp_bin(uint32_t* hist, bool active, uint32_t bin, int& binned,
+                                         unsigned* total) {
   if (active) atomicAdd(&hist[bin], 1u);
-  binned += __popc(__ballot_sync(0xFFFFFFFFu, active));
+  const int c = __popc(__ballot_sync(0xFFFFFFFFu, active));
+  binned += c;
+  if (c && (threadIdx.x & 31) == 0) atomicAdd(total, static_cast<unsigned>(c));
 }
 
 // Threshold K with exactly `need` keys >= K among keys[0..count) (count > need >= 1).
@@ -248,6 +251,7 @@ struct SelCtl {
   int abort_flag;
   int staged;
   int rank_bad;                // rank merge: the entries did not match the histogram
+  unsigned hist_total;         // candidates counted in `hist` this segment
   unsigned ref_ord[2];         // beam_step: max parent score (ordered) of a segment, by parity
   int wcount[32];
   int segoff[kMaxSegCounts + 1];
@@ -408,6 +412,7 @@ __device__ inline void cta_bitonic_desc(const Team& t, uint64_t* keys, int32_t* 
 // ------------------------------------------------------------ rank merge
 // Entries with values: nseg lists (list s holds count(s) entries).
 struct WarpListSrc {  // warp buffers in shared memory, stride cw
+  static constexpr bool kFlat = false;
   const uint64_t* keys;
   const int32_t* vals;
   int cw;
@@ -418,11 +423,22 @@ struct WarpListSrc {  // warp buffers in shared memory, stride cw
   __device__ __forceinline__ int32_t val(int s, int i) const { return vals[s * cw + i]; }
 };
 struct PartialListSrc {  // one request's partial lists in global memory, stride n
+  static constexpr bool kFlat = true;
   const unsigned long long* keys;
   const int32_t* vals;
   int n;
   const int* segoff;  // shared: list s holds segoff[s+1] - segoff[s] entries
   int nseg;
+  __device__ __forceinline__ int total() const { return segoff[nseg]; }
+  // Position in global memory of flat entry i (list found by binary search).
+  __device__ __forceinline__ size_t at(int i) const {
+    int lo = 0, hi = nseg;  // segoff[lo] <= i < segoff[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (segoff[mid] <= i) lo = mid; else hi = mid;
+    }
+    return static_cast<size_t>(lo) * n + (i - segoff[lo]);
+  }
   __device__ __forceinline__ int count(int s) const { return segoff[s + 1] - segoff[s]; }
   __device__ __forceinline__ uint64_t key(int s, int i) const {
     return __ldcg(keys + static_cast<size_t>(s) * n + i);
@@ -445,61 +461,93 @@ template <class Src, class Writer>
 __device__ bool rank_merge(const Team& t, SelCtl* ctl, const uint32_t* hist, const Src& src,
                            uint32_t n, int r, float C, uint64_t* stk, int32_t* stv, int cap,
                            uint32_t* P, uint32_t* cur, const Writer& out) {
-  // 1. Exclusive prefix counts, the bin bK of the n-th best and the work.
-  if (t.warp == 0) {
-    uint32_t carry = 0, work = 0;
-    int bK = -1;
-    for (int i = 0; i < kHistBins / 32; ++i) {
-      const int b = 32 * i + t.lane;
-      const uint32_t c = hist[b];
-      uint32_t incl = c;
+  // 1. Exclusive prefix counts P (each thread a contiguous chunk of bins),
+  //    the bin bK of the n-th best, and the in-bin compare work.
+  const int per = (kHistBins + t.T - 1) / t.T;
+  const int b0 = t.tid * per;
+  const int b1 = b0 + per < kHistBins ? b0 + per : kHistBins;
+  uint32_t mine = 0;
+  for (int b = b0; b < b1; ++b) mine += hist[b];
+  uint32_t incl = mine;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (t.lane >= o) incl += y;
-      }
-      const uint32_t excl = carry + incl - c;
-      P[b] = excl;
-      cur[b] = 0u;
-      if (bK < 0) {
-        const unsigned hit = __ballot_sync(0xFFFFFFFFu, excl + c >= n);
-        if (hit) bK = 32 * i + __ffs(hit) - 1;
-        const uint32_t cc = c < 4096u ? c : 4096u;
-        const uint32_t sq = (bK < 0 || b <= bK) ? cc * cc : 0u;
-        work += warp_sum_u(sq);
-      }
-      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-    }
-    if (bK < 0) bK = kHistBins - 1;  // fewer than n candidates: all of them rank
-    if (t.lane == 0) {
-      const uint32_t total = P[bK] + hist[bK];
-      ctl->bcast_d = bK;
-      ctl->bcast_cnt = total;
-      ctl->bcast_above = (total <= static_cast<uint32_t>(cap) && work <= kRankWorkLimit) ? 1u : 0u;
-      ctl->rank_bad = 0;
-    }
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (t.lane >= o) incl += y;
+  }
+  if (t.lane == 31) ctl->red[t.warp] = incl;
+  if (t.tid == 0) {
+    ctl->bcast_d = kHistBins;
+    ctl->bcast_cnt = 0u;
+    ctl->rank_bad = 0;
   }
   team_sync(t);
-  if (!ctl->bcast_above) return false;
-  const int bK = ctl->bcast_d;
-  const int total = static_cast<int>(ctl->bcast_cnt);
-  for (int i = t.tid; i < total; i += t.T) stk[i] = 0ull;
+  uint32_t base = incl - mine;
+  for (int w = 0; w < t.warp; ++w) base += static_cast<uint32_t>(ctl->red[w]);
+  for (int b = b0; b < b1; ++b) {
+    const uint32_t c = hist[b];
+    P[b] = base;
+    cur[b] = 0u;
+    if (base + c >= n) {
+      atomicMin(&ctl->bcast_d, b);
+      break;  // the bins after this one are below bK: never needed
+    }
+    base += c;
+  }
+  team_sync(t);
+  int bK = ctl->bcast_d;
+  if (bK >= kHistBins) bK = kHistBins - 1;  // fewer than n candidates: all of them rank
+  {
+    uint32_t work = 0;
+    for (int b = b0; b < b1 && b <= bK; ++b) {
+      const uint32_t c = hist[b] < 4096u ? hist[b] : 4096u;
+      work += c * c;
+    }
+    work = warp_sum_u(work);
+    if (t.lane == 0 && work) atomicAdd(&ctl->bcast_cnt, work);
+  }
+  team_sync(t);
+  const uint32_t total = P[bK] + hist[bK];
+  if (total > static_cast<uint32_t>(cap) || ctl->bcast_cnt > kRankWorkLimit) return false;
+  for (int i = t.tid; i < static_cast<int>(total); i += t.T) stk[i] = 0ull;
   team_sync(t);
   // 2. Scatter the entries of bins 0..bK into their bins' slot ranges.
-  for (int s = 0; s < src.nseg; ++s) {
-    const int c = src.count(s);
-    for (int i = t.tid; i < c; i += t.T) {
-      const uint64_t key = src.key(s, i);
-      if (key == 0ull) continue;
-      const uint32_t b = score_bin(key_score(key), C);
-      if (b > static_cast<uint32_t>(bK)) continue;
-      const uint32_t slot = P[b] + atomicAdd(&cur[b], 1u);
-      if (slot < P[b] + hist[b]) {
-        stk[slot] = key;
-        stv[slot] = src.val(s, i);
-      } else {
-        ctl->rank_bad = 1;
+  auto place = [&](uint64_t key, int32_t val) {
+    if (key == 0ull) return;
+    const uint32_t b = score_bin(key_score(key), C);
+    if (b > static_cast<uint32_t>(bK)) return;
+    const uint32_t slot = P[b] + atomicAdd(&cur[b], 1u);
+    if (slot < P[b] + hist[b]) {
+      stk[slot] = key;
+      stv[slot] = val;
+    } else {
+      ctl->rank_bad = 1;
+    }
+  };
+  if constexpr (Src::kFlat) {
+    // Global lists: eight independent loads per thread before any use.
+    constexpr int kU = 8;
+    const int M = src.total();
+    for (int base_i = 0; base_i < M; base_i += kU * t.T) {
+      uint64_t key[kU];
+      int32_t val[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = base_i + u * t.T + t.tid;
+        key[u] = 0ull;
+        val[u] = -1;
+        if (i < M) {
+          const size_t at = src.at(i);
+          key[u] = __ldcg(src.keys + at);
+          val[u] = __ldcg(src.vals + at);
+        }
       }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) place(key[u], val[u]);
+    }
+  } else {
+    for (int s = 0; s < src.nseg; ++s) {
+      const int c = src.count(s);
+      for (int i = t.tid; i < c; i += t.T) place(src.key(s, i), src.val(s, i));
     }
   }
   team_sync(t);
@@ -645,7 +693,8 @@ __device__ __forceinline__ void warp_offer(WarpBuf& wb, bool valid, uint64_t key
 // keep an L2 round trip off this path). Warp-collective.
 __device__ __forceinline__ void refresh_thr(WarpBuf& wb, SelCtl* ctl, uint32_t n, float C,
                                             int lane, const ThrSinks& sinks) {
-  if (wb.binned < kRefreshAfter && wb.thr != 0ull) {
+  if ((wb.binned < kRefreshAfter && wb.thr != 0ull) ||
+      *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) < n) {
     const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
     if (c > wb.thr) wb.thr = c;
     return;
@@ -670,8 +719,9 @@ struct FlushArgs {
   int k;                  // this CTA's contributor index for request r
   int G;                  // contributors of request r
   int maxG;               // partial-list slots per request
-  unsigned long long* part_keys;  // [R][maxG][n]
-  int32_t* part_vals;             // [R][maxG][n]
+  int pcap;               // capacity (and stride) of one partial list
+  unsigned long long* part_keys;  // [R][maxG][pcap]
+  int32_t* part_vals;             // [R][maxG][pcap]
   uint32_t* part_count;           // [R][maxG]
   uint32_t* tickets;              // [R]
   unsigned long long* request_thr;  // [R]
@@ -712,7 +762,7 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
   for (int i = t.tid; i < kHistBins; i += t.T) ctl->hist[i] = __ldcg(gh + i);
   for (int k = t.tid; k < G; k += t.T) {
     const int c = static_cast<int>(__ldcg(f.part_count + list0 + k));
-    ctl->segoff[k + 1] = c < f.n ? c : f.n;
+    ctl->segoff[k + 1] = c < f.pcap ? c : f.pcap;
   }
   team_sync(t);
   if (t.warp == 0) {  // exclusive prefix sum of the list sizes
@@ -735,6 +785,22 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
     }
   }
   team_sync(t);
+  {
+    const unsigned long long* lists0 = f.part_keys + list0 * f.pcap;
+    const int32_t* lvals0 = f.part_vals + list0 * f.pcap;
+    if (f.rank_P &&
+        rank_merge(t, ctl, ctl->hist, PartialListSrc{lists0, lvals0, f.pcap, ctl->segoff, G},
+                   static_cast<uint32_t>(f.n), f.r, f.C, f.sort_keys, f.sort_vals, f.sort_cap,
+                   f.rank_P, f.rank_cur, out)) {
+      for (int i = t.tid; i < kHistBins; i += t.T) gh[i] = 0u;
+      if (t.tid == 0) {
+        f.tickets[f.r] = 0u;
+        f.request_thr[f.r] = 0ull;
+      }
+      return;
+    }
+  }
+  team_sync(t);
   if (t.warp == 0) {
     const uint64_t hb = hist_bound(ctl->hist, static_cast<uint32_t>(f.n), f.C, t.lane);
     if (t.lane == 0) {
@@ -746,19 +812,8 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
   team_sync(t);
   const uint64_t K0 = ctl->bcast_key;
   const int total = ctl->segoff[G];
-  const unsigned long long* lists = f.part_keys + list0 * f.n;
-  const int32_t* lvals = f.part_vals + list0 * f.n;
-  if (f.rank_P &&
-      rank_merge(t, ctl, ctl->hist, PartialListSrc{lists, lvals, f.n, ctl->segoff, G},
-                 static_cast<uint32_t>(f.n), f.r, f.C, f.sort_keys, f.sort_vals, f.sort_cap,
-                 f.rank_P, f.rank_cur, out)) {
-    for (int i = t.tid; i < kHistBins; i += t.T) gh[i] = 0u;
-    if (t.tid == 0) {
-      f.tickets[f.r] = 0u;
-      f.request_thr[f.r] = 0ull;
-    }
-    return;
-  }
+  const unsigned long long* lists = f.part_keys + list0 * f.pcap;
+  const int32_t* lvals = f.part_vals + list0 * f.pcap;
   // Filtered copy of all partial entries >= K0 into [0, cap): flat index,
   // segment found by binary search, four independent loads per thread.
   uint64_t* stk = f.sort_keys;
@@ -780,7 +835,7 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
           const int mid = (lo + hi) >> 1;
           if (ctl->segoff[mid] <= i) lo = mid; else hi = mid;
         }
-        const size_t at = static_cast<size_t>(lo) * f.n + (i - ctl->segoff[lo]);
+        const size_t at = static_cast<size_t>(lo) * f.pcap + (i - ctl->segoff[lo]);
         key[u] = __ldcg(lists + at);
         val[u] = __ldcg(lvals + at);
       }
@@ -806,7 +861,7 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
     while (N_all < sel_all) N_all <<= 1;
     uint64_t Kg = 0;
     if (M > f.n)
-      Kg = cta_select(t, PartialSrc{lists, f.n, ctl->segoff, G}, f.n, f.radix_hist, ctl);
+      Kg = cta_select(t, PartialSrc{lists, f.pcap, ctl->segoff, G}, f.n, f.radix_hist, ctl);
     if (t.tid == 0) ctl->counter = 0;
     for (int i = t.tid; i < N_all; i += t.T) {
       stk[i] = 0ull;
@@ -823,7 +878,7 @@ __device__ void request_merge(const Team& t, SelCtl* ctl, const FlushArgs& f, co
           const int mid = (lo + hi) >> 1;
           if (ctl->segoff[mid] <= i) lo = mid; else hi = mid;
         }
-        const size_t at = static_cast<size_t>(lo) * f.n + (i - ctl->segoff[lo]);
+        const size_t at = static_cast<size_t>(lo) * f.pcap + (i - ctl->segoff[lo]);
         key = __ldcg(lists + at);
         val = __ldcg(lvals + at);
       }
@@ -939,6 +994,7 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
     wb.thr = 0;
     if (t.tid == 0) {
       ctl->cta_thr = 0ull;
+      ctl->hist_total = 0u;
       f.request_thr[f.r] = 0ull;
     }
     team_sync(t);
@@ -976,7 +1032,7 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
     if (t.lane == 0 && ge) atomicAdd(&ctl->counter, ge);
   }
   team_sync(t);
-  if (ctl->counter > f.n) {
+  if (ctl->counter > f.pcap) {  // more survivors than the list holds: keep the n best
     const uint64_t Kc = cta_select(t, WarpBufSrc{f.wkeys, f.cw, ctl->wcount, t.nwarps}, f.n,
                                    f.radix_hist, ctl);
     if (Kc > K) K = Kc;
@@ -985,12 +1041,12 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
   team_sync(t);
   if (t.tid == 0) ctl->counter = 0;
   team_sync(t);
-  const size_t slot = (static_cast<size_t>(f.r) * f.maxG + f.k) * f.n;
+  const size_t slot = (static_cast<size_t>(f.r) * f.maxG + f.k) * f.pcap;
   for (int base = 0; base < wb.count; base += 32) {
     const int i = base + t.lane;
     const bool keep = i < wb.count && wb.keys[i] >= K;
     const int pos = append_pos(&ctl->counter, keep, t.lane);
-    if (keep && pos < f.n) {
+    if (keep && pos < f.pcap) {
       f.part_keys[slot + pos] = wb.keys[i];
       f.part_vals[slot + pos] = wb.vals[i];
     }
@@ -999,7 +1055,7 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
   team_sync(t);
   // 3. Ticket; the last contributor merges the request.
   if (t.tid == 0) {
-    const int c = ctl->counter < f.n ? ctl->counter : f.n;
+    const int c = ctl->counter < f.pcap ? ctl->counter : f.pcap;
     f.part_count[static_cast<size_t>(f.r) * f.maxG + f.k] = static_cast<uint32_t>(c);
     __threadfence();
     const unsigned tk = atomicAdd(f.tickets + f.r, 1u);
@@ -1015,7 +1071,10 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
   for (int i = t.tid; i < kHistBins; i += t.T) ctl->hist[i] = 0u;
   wb.count = 0;
   wb.thr = 0;
-  if (t.tid == 0) ctl->cta_thr = 0ull;
+  if (t.tid == 0) {
+    ctl->cta_thr = 0ull;
+    ctl->hist_total = 0u;
+  }
   team_sync(t);
   return false;
 }
