@@ -169,24 +169,20 @@ def run_ours(args, world, rank, local):
             b += live_rows[t] * mask_row
         step_bytes.append(b)
 
-    def one_search(i, ev=None):
-        lset = sets[i % len(sets)]
-        for t in range(w.depth):
-            if ev is not None:
-                ev[t][0].record(stream)
-            search.step(t, lset[t], stream=stream)
-            if ev is not None:
-                ev[t][1].record(stream)
-        search.finalize(stream=stream)
-
+    # 2. One CUDA graph per logits copy (five beam_step launches + finalize);
+    #    the timed region replays them in rotation. A second set of graphs with
+    #    events between the launches gives each step's device time.
+    graphs = [search.capture(sets[i]) for i in range(len(sets))]
+    ev_sets = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(w.depth + 2)]
+               for _ in range(len(sets))]
+    ev_graphs = [search.capture(sets[i], events=ev_sets[i]) for i in range(len(sets))]
+    torch.cuda.synchronize()
     for i in range(args.warmup):
-        one_search(i)
+        graphs[i % len(graphs)].replay()
     torch.cuda.synchronize()
     assert torch.equal(search.sids, ref_sids), "replay diverged from the generated search"
 
     K = args.steps
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-            for _ in range(w.depth)] for _ in range(K)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
         if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, "/tmp/_clk.csv")
@@ -196,7 +192,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     start.record(stream)
     for i in range(K):
-        one_search(i, evs[i])
+        graphs[i % len(graphs)].replay()
     stop.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -210,8 +206,20 @@ def run_ours(args, world, rank, local):
     assert torch.equal(search.sids, ref_sids)
     assert tcb.sidbeam_get_device_status(search.workspace) == 0
 
-    per_step_us = [statistics.mean(evs[i][t][0].elapsed_time(evs[i][t][1]) for i in range(K)) * 1e3
-                   for t in range(w.depth)]
+    # Per-step device times (graph replays with events, outside the timed region).
+    reps = max(30, min(300, K // 4))
+    acc = [[0.0] * (w.depth + 1) for _ in range(len(sets))]
+    cnt = [0] * len(sets)
+    for i in range(reps):
+        j = i % len(sets)
+        ev_graphs[j].replay()
+        torch.cuda.synchronize()
+        ev = ev_sets[j]
+        for t in range(w.depth + 1):
+            acc[j][t] += ev[t].elapsed_time(ev[t + 1])
+        cnt[j] += 1
+    per_step_us = [1e3 * sum(acc[j][t] for j in range(len(sets))) / sum(cnt) for t in range(w.depth)]
+    finalize_us = 1e3 * sum(acc[j][w.depth] for j in range(len(sets))) / sum(cnt)
     steady = list(range(1, w.depth))
     dur_us = statistics.mean(per_step_us[t] for t in steady)
     bytes_launch = statistics.mean(step_bytes[t] for t in steady)
@@ -219,7 +227,7 @@ def run_ours(args, world, rank, local):
     achieved = bytes_launch / (dur_us * 1e-6) / 1e9
     value = world * K * logits_per_search / (elapsed_ms * 1e-3)
 
-    # 2. End to end through the C ABI with host buffers: per search, copy every
+    # 3. End to end through the C ABI with host buffers: per search, copy every
     #    step's logits from pinned host memory, run, copy the results back.
     e2e = None
     if not args.no_e2e:
@@ -263,7 +271,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds, cat=cat)
 
     traffic = _profile_traffic()
     line = {
@@ -277,6 +285,9 @@ def run_ours(args, world, rank, local):
                      "kernel": "beam_step_kernel<bf16>, steady steps 1-4",
                      "bytes_per_launch": bytes_launch, "us_per_launch": dur_us},
         "step_us": per_step_us,
+        "finalize_us": finalize_us,
+        "timing": "CUDA graph replays of the whole search (5 beam_step + beam_finalize), "
+                  "3 rotating logits copies; per-step times from events inside the graph",
         "logits_per_step": logits_per_search,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -310,31 +321,34 @@ def _oracle_inputs(w, base, search, t):
     return lg, ps.cpu().numpy(), pn.cpu().numpy(), B_in
 
 
-def _oracle_trie(w):
+def _oracle_trie(w, cat=None):
     import oracle
-    return oracle.OracleTrie(w.catalog(), w.codes_per_level)
+    return oracle.OracleTrie(w.catalog() if cat is None else cat, w.codes_per_level)
 
 
-def cpu_baseline(w, base, search, live_rows, budget_s=15.0, trie=None):
-    """Time the oracle's beam step on a bounded sample of steady step 2
-    (whole requests of 512 rows x 4,096 bf16 logits) on this host's cores."""
+def cpu_baseline(w, base, search, live_rows, budget_s=15.0, trie=None, cat=None):
+    """Time the oracle's beam step on a bounded sample of the same search: whole
+    requests (512 rows x 4,096 bf16 logits) of steps 1-4 in turn, until the
+    budget is spent, on this host's cores."""
     import oracle
-    trie = trie or _oracle_trie(w)
-    t = 2
-    lg, ps, pn, B_in = _oracle_inputs(w, base, search, t)
+    trie = trie or _oracle_trie(w, cat)
+    inputs = {t: _oracle_inputs(w, base, search, t) for t in range(1, w.depth)}
+    order = [(t, r) for r in range(w.R) for t in range(1, w.depth)]
     done_rows = 0
-    reqs = 0
+    calls = 0
     t0 = time.perf_counter()
-    while reqs < w.R and time.perf_counter() - t0 < budget_s:
-        sl = slice(reqs * B_in, (reqs + 1) * B_in)
+    while calls == 0 or time.perf_counter() - t0 < budget_s:
+        t, r = order[calls % len(order)]
+        lg, ps, pn, B_in = inputs[t]
+        sl = slice(r * B_in, (r + 1) * B_in)
         oracle.beam_step(trie, t, lg[sl], ps[sl], pn[sl], 1, B_in, w.n, w.V)
         done_rows += int(np.isfinite(ps[sl]).sum())
-        reqs += 1
+        calls += 1
     el = time.perf_counter() - t0
     return {"value": done_rows * w.V / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"oracle.beam_step on {reqs} request(s) of step {t} "
-                      f"({B_in} rows x {w.V} bf16 logits each), {el:.1f} s, numpy float64, "
-                      f"single thread; host has {os.cpu_count()} cores"}
+            "sample": f"oracle.beam_step on {calls} whole requests of steps 1-{w.depth - 1} "
+                      f"(512 rows x {w.V} bf16 logits each, steps in turn), {el:.1f} s, numpy "
+                      f"float64, single thread; host has {os.cpu_count()} cores"}
 
 
 # ----------------------------------------------------------------- reference arm

@@ -727,6 +727,49 @@ __device__ __forceinline__ float segment_ref(const StepArgs& a, const Team& t, S
   return o ? unord_f32(o) : 0.f;
 }
 
+// --------------------------------------------------------------- segment end
+// Once per segment, out of line (away from the per-row loop). The warp buffer
+// goes in by value so that the caller's copy stays in registers; the caller
+// empties its own copy afterwards.
+__device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf wb, SelCtl* ctl,
+                                         uint64_t* wkeys, int32_t* wvals, uint32_t* whist,
+                                         uint32_t* cta_hist, uint8_t* stages, int direct_cap,
+                                         int cur_r, int r_last, float C) {
+  const StepConfig& cfg = a.cfg;
+  FlushArgs f;
+  f.n = a.n;
+  f.r = cur_r;
+  f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
+  f.G = a.part.contributors(cur_r);
+  f.maxG = a.part.maxG;
+  f.pcap = partial_cap(a.n);
+  f.part_keys = a.part_keys;
+  f.part_vals = a.part_vals;
+  f.part_count = a.part_count;
+  f.tickets = a.tickets;
+  f.request_thr = a.request_thr;
+  f.ghist = a.ghist;
+  f.C = C;
+  f.wkeys = wkeys;
+  f.cw = cfg.Cw;
+  f.sort_keys = wkeys;
+  f.sort_vals = wvals;
+  f.sort_cap = cfg.W * cfg.Cw;
+  f.radix_hist = cta_hist;
+  f.wvals = wvals;
+  f.rank_P = whist;
+  f.rank_cur = whist + kHistBins;
+  // The stages are idle only at the CTA's last segment (every ring is empty).
+  const bool last = cur_r == r_last;
+  f.direct_keys = last ? reinterpret_cast<uint64_t*>(stages) : nullptr;
+  f.direct_vals =
+      last ? reinterpret_cast<int32_t*>(stages + static_cast<size_t>(direct_cap) * 8) : nullptr;
+  f.direct_cap = last ? direct_cap : 0;
+  const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
+                          static_cast<uint32_t>(a.V)};
+  return segment_flush(team, wb, ctl, f, writer);
+}
+
 // --------------------------------------------------------------- kernel
 template <int BF16, int REG>
 __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 32, 1)
@@ -831,43 +874,16 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
              wvals + static_cast<size_t>(warp) * cfg.Cw, whist + warp * 256, cfg.Cw, 0, 0ull, 0};
   uint32_t* my_prefix = wprefix + warp * cfg.prefix_words;
   uint32_t* my_mask = wmask + warp * cfg.prefix_words;
-  const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
-                          static_cast<uint32_t>(a.V)};
   const int direct_cap = (W * S * cfg.stage_bytes / 12) & ~1;
 
   // End of the segment of request cur_r (all warps, in the same order).
   int cur_r = r_first;
   auto flush = [&]() -> bool {
-    FlushArgs f;
-    f.n = a.n;
-    f.r = cur_r;
-    f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
-    f.G = a.part.contributors(cur_r);
-    f.maxG = a.part.maxG;
-    f.pcap = partial_cap(a.n);
-    f.part_keys = a.part_keys;
-    f.part_vals = a.part_vals;
-    f.part_count = a.part_count;
-    f.tickets = a.tickets;
-    f.request_thr = a.request_thr;
-    f.ghist = a.ghist;
-    f.C = C;
-    f.wkeys = wkeys;
-    f.cw = cfg.Cw;
-    f.sort_keys = wkeys;
-    f.sort_vals = wvals;
-    f.sort_cap = W * cfg.Cw;
-    f.radix_hist = cta_hist;
-    f.wvals = wvals;
-    f.rank_P = whist;
-    f.rank_cur = whist + kHistBins;
-    // The stages are idle only at the CTA's last segment (every ring is empty).
-    const bool last = cur_r == r_last;
-    f.direct_keys = last ? reinterpret_cast<uint64_t*>(stages) : nullptr;
-    f.direct_vals = last ? reinterpret_cast<int32_t*>(stages + static_cast<size_t>(direct_cap) * 8)
-                         : nullptr;
-    f.direct_cap = last ? direct_cap : 0;
-    if (segment_flush(team, wb, ctl, f, writer)) return true;
+    const bool stop = segment_end(a, team, wb, ctl, wkeys, wvals, whist, cta_hist, stages,
+                                  direct_cap, cur_r, r_last, C);
+    wb.count = 0;
+    wb.thr = 0ull;
+    if (stop) return true;
     if (cur_r < r_last) C = segment_ref(a, team, ctl, cur_r + 1, ref_slot ^= 1);
     ++cur_r;
     return false;

@@ -52,6 +52,31 @@ class BeamSearch:
                              self.nodes[self.depth - 1], self.sids, self.leaf, stream=stream)
         return self.sids, self.leaf, self.scores[self.depth - 1].view(self.R, self.n)
 
+    def capture(self, logits_per_step, events=None):
+        """A CUDA graph of the whole search (every beam_step, then beam_finalize)
+        on fixed logits tensors; ``graph.replay()`` runs it on the current stream.
+
+        Call the search once eagerly first (that sets the kernels' shared-memory
+        limits outside the capture). ``events``: optional depth + 2 events made
+        with ``enable_timing=True, external=True``, recorded before every step,
+        before finalize and at the end (per-step device times of a replay).
+        """
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=side):
+            for t in range(self.depth):
+                if events is not None:
+                    events[t].record()
+                self.step(t, logits_per_step[t])
+            if events is not None:
+                events[self.depth].record()
+            self.finalize()
+            if events is not None:
+                events[self.depth + 1].record()
+        torch.cuda.current_stream().wait_stream(side)
+        return g
+
     def run(self, logits_for_step, stream=None):
         """logits_for_step(t, search) -> logits tensor [rows(t), ld] for step t."""
         for t in range(self.depth):
