@@ -138,8 +138,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
 
     # 1. Generate the search's logits once (generator keyed by prefix hash).
-    hashes = torch.full((w.R,), int(np.uint64(host.PREFIX_HASH_SEED).view(np.int64)),
-                        dtype=torch.int64, device=dev)
+    hashes = torch.from_numpy(host.request_roots(w.R).view(np.int64)).to(dev)
     base = []
     live_rows = []
     for t in range(w.depth):

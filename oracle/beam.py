@@ -121,8 +121,9 @@ def beam_finalize(bp_parent, bp_code, last_score, last_node):
 def beam_search(trie, R: int, n: int, depth: int, V: int, logits_for_rows):
     """Full constrained beam search from the root.
 
-    logits_for_rows(step, prefixes) -> logits [rows, V] for the given live
-    prefixes (int array [rows, step]); dead rows are never asked for.
+    logits_for_rows(step, prefixes, requests) -> logits [rows, V] for the given
+    live prefixes (int array [rows, step]) of the given requests (int array
+    [rows]); dead rows are never asked for.
     Returns finalize's dict plus per-step outputs (``steps``).
     """
     parent_scores = np.zeros(R)                    # step 0: one root row per request
@@ -136,7 +137,8 @@ def beam_search(trie, R: int, n: int, depth: int, V: int, logits_for_rows):
         flat_live = np.flatnonzero(live.reshape(-1))
         if flat_live.size:
             logits[flat_live] = _widen(
-                logits_for_rows(t, prefixes.reshape(R * B_in, t)[flat_live]))[:, :V]
+                logits_for_rows(t, prefixes.reshape(R * B_in, t)[flat_live],
+                                flat_live // B_in))[:, :V]
         out = beam_step(trie, t, logits, parent_scores, parent_nodes, R, B_in, n, V)
         steps.append(out)
         new_prefixes = np.full((R, n, t + 1), -1, dtype=np.int64)

@@ -27,6 +27,7 @@ from .host import (  # noqa: F401
     normal_from_counters,
     philox4x32_10,
     prefix_hashes,
+    request_roots,
     row_logits,
     table_logits,
     hidden_states,

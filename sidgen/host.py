@@ -38,8 +38,10 @@ GOLDEN_GAMMA = 0x9E3779B97F4A7C15
 _SM_C1 = np.uint64(0xBF58476D1CE4E5B9)
 _SM_C2 = np.uint64(0x94D049BB133111EB)
 
-# Hash of the empty prefix (the trie root): the first 64 bits of pi's
-# fractional part, a nothing-up-my-sleeve constant.
+# Seed of the prefix-hash chain: the first 64 bits of pi's fractional part, a
+# nothing-up-my-sleeve constant. Request r's empty prefix (its trie root) hashes
+# to mix(PREFIX_HASH_SEED ^ r): each request stands for its own context, so
+# concurrent requests search different logits.
 PREFIX_HASH_SEED = 0x243F6A8885A308D3
 
 # Counter word 3 separates the independent streams that one seed feeds.
@@ -80,8 +82,16 @@ def splitmix64_stream(seed: int, start: int, count: int) -> np.ndarray:
     return splitmix64_mix(state)
 
 
-def root_hash() -> np.uint64:
-    return np.uint64(PREFIX_HASH_SEED)
+def root_hash(request=0):
+    """Hash of request ``request``'s empty prefix (scalar or array of requests)."""
+    r = _u64(request)
+    h = splitmix64_mix(_u64(PREFIX_HASH_SEED) ^ r)
+    return h if h.ndim else np.uint64(h)
+
+
+def request_roots(R: int) -> np.ndarray:
+    """Root hashes of requests 0 .. R-1 (uint64 [R])."""
+    return root_hash(np.arange(R, dtype=np.uint64))
 
 
 def child_hash(parent_hash, level: int, code) -> np.ndarray:
@@ -90,11 +100,15 @@ def child_hash(parent_hash, level: int, code) -> np.ndarray:
     return splitmix64_mix(_u64(parent_hash) ^ tag)
 
 
-def prefix_hashes(prefixes: np.ndarray) -> np.ndarray:
-    """Hashes of an array of prefixes [rows, l] (l may be 0)."""
+def prefix_hashes(prefixes: np.ndarray, requests=None) -> np.ndarray:
+    """Hashes of an array of prefixes [rows, l] (l may be 0) of the given
+    requests (int array [rows]; all request 0 when omitted)."""
     prefixes = np.asarray(prefixes)
     rows = prefixes.shape[0]
-    h = np.full(rows, PREFIX_HASH_SEED, dtype=np.uint64)
+    if requests is None:
+        h = np.full(rows, root_hash(0), dtype=np.uint64)
+    else:
+        h = root_hash(np.asarray(requests, dtype=np.uint64).reshape(rows))
     for lv in range(prefixes.shape[1]):
         h = child_hash(h, lv + 1, prefixes[:, lv].astype(np.uint64))
     return h

@@ -4,7 +4,9 @@ They stand in for the pages' workloads (RecIF-Bench / OneRec traffic, Sohu
 traffic, Amazon/Yelp catalogs), none of which is available: SID depth 3-5,
 codebooks of 256-8192 codes, beam widths 8-512 across concurrent requests,
 catalogs from thousands to millions of SIDs. Seeds: catalog 1000*c + 1,
-logits / hidden states 1000*c + 2, lm_head weight 1000*c + 3.
+logits / hidden states 1000*c + 2, lm_head weight 1000*c + 3. Every request's
+prefix-hash chain starts from its own root (``host.request_roots``), so concurrent
+requests search different logits.
 """
 from __future__ import annotations
 

@@ -100,8 +100,7 @@ def run_gpu_search(trie_gpu, R, n, depth, V, seed, sigma, dtype, ld_pad=0, on_st
     from sidgen import device as gdev
 
     search = tcb.BeamSearch(trie_gpu, R, n, V, depth=depth)
-    hashes = torch.full((R,), np.int64(np.uint64(host.PREFIX_HASH_SEED).view(np.int64)),
-                        dtype=torch.int64, device="cuda")
+    hashes = torch.from_numpy(host.request_roots(R).view(np.int64)).to("cuda")
     tdt = torch.float32 if dtype == "f32" else torch.bfloat16
     elem = 4 if dtype == "f32" else 2
     for t in range(depth):
@@ -137,8 +136,9 @@ def oracle_search_with_gaps(trie, R, n, depth, V, seed, sigma, dtype):
     """Oracle search (host generator) that also reports, per request, the smallest
     gap over steps between the n-th and the (n+1)-th candidate: a near-tie there
     changes the beam set, so end-to-end parity is only defined where it is wide."""
-    def fn(step, prefixes):
-        return host.row_logits(seed, host.prefix_hashes(prefixes), V, sigma, dtype=dtype)
+    def fn(step, prefixes, requests):
+        return host.row_logits(seed, host.prefix_hashes(prefixes, requests), V, sigma,
+                               dtype=dtype)
 
     scores = np.zeros(R)
     nodes = np.zeros(R, dtype=np.int64)
@@ -151,7 +151,7 @@ def oracle_search_with_gaps(trie, R, n, depth, V, seed, sigma, dtype):
         live = np.flatnonzero(scores > -np.inf)
         z = np.zeros((R * B_in, V))
         if live.size:
-            z[live] = _widen(fn(t, flat[live]))
+            z[live] = _widen(fn(t, flat[live], live // B_in))
         ext = oracle.beam_step(trie, t, z, scores, nodes, R, B_in, n + 1, V)
         sc = ext["score"]
         for r in range(R):   # boundary gap: n-th kept vs first left out

@@ -58,7 +58,14 @@ def test_prefix_hash_chains():
     manual = host.child_hash(host.child_hash(host.child_hash(host.root_hash(), 1, 3), 2, 5), 3, 7)
     assert int(h[0]) == int(manual)
     assert h[0] != h[1]
-    assert int(host.prefix_hashes(np.zeros((1, 0), dtype=np.int64))[0]) == host.PREFIX_HASH_SEED
+    empty = np.zeros((3, 0), dtype=np.int64)
+    assert int(host.prefix_hashes(empty)[0]) == int(host.root_hash(0))
+    roots = host.prefix_hashes(empty, np.array([0, 1, 2]))
+    assert len({int(x) for x in roots}) == 3          # requests start from distinct roots
+    assert int(roots[2]) == int(host.splitmix64_mix(np.uint64(host.PREFIX_HASH_SEED ^ 2)))
+    h1 = host.prefix_hashes(pre, np.array([1, 1]))
+    assert int(h1[0]) == int(host.child_hash(host.child_hash(host.child_hash(
+        host.root_hash(1), 1, 3), 2, 5), 3, 7))
 
 
 def test_catalog_draw_distinct_and_in_range():

@@ -23,8 +23,8 @@ from sidgen import host
 
 
 def _gen_logits_fn(seed, V, sigma):
-    def fn(step, prefixes):
-        return host.row_logits(seed, host.prefix_hashes(prefixes), V, sigma)
+    def fn(step, prefixes, requests=None):
+        return host.row_logits(seed, host.prefix_hashes(prefixes, requests), V, sigma)
     return fn
 
 
@@ -96,8 +96,8 @@ def test_exhaustive_equals_beam_search_random_tiny(case):
     V = max(Vs)
     fn = _gen_logits_fn(77 + case, V, 1.7)
 
-    def fn_level(step, prefixes):   # per-level codebook: only the first V_l codes exist
-        return fn(step, prefixes)[:, :Vs[step]]
+    def fn_level(step, prefixes, requests=None):  # per-level codebook: first V_l codes only
+        return fn(step, prefixes, requests)[:, :Vs[step]]
 
     R = 1
     n = n_cat + int(rng.integers(0, 4))
@@ -293,7 +293,7 @@ def test_catalog_scorer_equals_beam_search_prefix_independent():
     lp = np.stack([[oracle.log_softmax_full(table[r, lv]) for lv in range(3)] for r in range(R)])
     sc = oracle.catalog_score_topk(trie, lp, K)
     for r in range(R):
-        def fn(step, prefixes, r=r):    # logits depend on the level only, not the prefix
+        def fn(step, prefixes, requests, r=r):  # logits depend on the level only
             return np.repeat(table[r, step][None], prefixes.shape[0], axis=0)
         bs = oracle.beam_search(trie, 1, 500, 3, 16, fn)
         assert bs["leaf"][0, :K].tolist() == sc["leaf"][r].tolist()

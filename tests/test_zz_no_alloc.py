@@ -39,8 +39,7 @@ def test_noalloc_matches_workspace_path_two_calls(tcb):
     R, n = 8, 32
     cat = w.catalog()
     trie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
-    hashes = torch.full((R,), int(np.uint64(host.PREFIX_HASH_SEED).view(np.int64)),
-                        dtype=torch.int64, device="cuda")
+    hashes = torch.from_numpy(host.request_roots(R).view(np.int64)).to("cuda")
     ps = torch.zeros(R, dtype=torch.float32, device="cuda")
     pn = torch.zeros(R, dtype=torch.int32, device="cuda")
     B_in = 1

@@ -45,9 +45,9 @@ using namespace dev;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRegVecs = 16;  // 16-byte vectors per lane held in registers (8 KB rows)
-// Dense rows with more children than this (per warp taking part) are walked in
-// place in their stage, in two passes, instead of from registers.
-constexpr uint32_t kHeavyDense = 128;
+// A register row with more hits than this is walked in two passes (count,
+// raise the threshold, offer).
+constexpr int kOnePassHits = 64;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // f(I) for I = 0 .. N-1 with I a compile-time constant (keeps register arrays
@@ -575,13 +575,15 @@ __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRe
   return __any_sync(kFull, (hp[0] | hp[1] | hp[2] | hp[3]) != 0u);
 }
 
-// Counts every hit in the CTA histogram and offers it to the warp buffer (one
-// pass; a hit that falls below a threshold raised meanwhile is dropped). The
-// logits of the hits are read again from the row in global memory (it was
-// just streamed, so from L2): four per lane per round trip, one compact loop
-// instead of a copy of the walk per register vector.
-template <int BF16>
-__device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* grow,
+// Counts the hits in the CTA histogram and/or offers them to the warp buffer
+// (MODE); when offering, a hit that falls below a threshold raised meanwhile
+// is dropped. The logits of the hits are read from the row's stage (held
+// until the walk is done): one compact loop instead of a copy of the walk per
+// register vector.
+enum TakeMode { kTakeBinOffer = 0, kTakeBin = 1, kTakeOffer = 2 };
+
+template <int BF16, int MODE>
+__device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* zrow,
                                           const uint32_t (&hp)[kRegVecs / 4],
                                           const uint32_t* wmask, uint32_t* wprefix,
                                           const RowCtx& c, float& zthr, WarpBuf& wb, SelCtl* ctl,
@@ -589,7 +591,7 @@ __device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* grow
   constexpr int kPerVec = BF16 ? 8 : 4;
   constexpr int kBatch = 4;
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  if (dense) dense_prefix(wmask, a.mask_words, wprefix, lane);
+  if (dense && MODE != kTakeBin) dense_prefix(wmask, a.mask_words, wprefix, lane);
   uint32_t hb[kRegVecs / 4] = {hp[0], hp[1], hp[2], hp[3]};
   while (__any_sync(kFull, (hb[0] | hb[1] | hb[2] | hb[3]) != 0u)) {
     int code[kBatch];
@@ -604,61 +606,101 @@ __device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* grow
       code[u] = bit < 0 ? -1 : (lane + 32 * (bit >> 3)) * kPerVec + (bit & 7);
     }
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      z[u] = 0.f;
-      if (code[u] >= 0) {
-        if (BF16)
-          z[u] = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short*>(grow) + code[u])) << 16);
-        else
-          z[u] = __ldg(reinterpret_cast<const float*>(grow) + code[u]);
-      }
-    }
+    for (int u = 0; u < kBatch; ++u) z[u] = code[u] >= 0 ? elem<BF16>(zrow, code[u]) : 0.f;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const bool has = code[u] >= 0 && z[u] >= zthr;
+      const bool has = code[u] >= 0 && (MODE == kTakeBin || z[u] >= zthr);
       if (!__any_sync(kFull, has)) continue;
       const float score = c.s + (z[u] - c.lse);
-      warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
-      const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code[u]) : -1;
-      warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code[u])), node,
-                    static_cast<uint32_t>(a.n), lane, sinks);
-      zthr = zthreshold(wb.thr, c.s, c.lse);
+      if (MODE != kTakeOffer)
+        warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
+      if (MODE != kTakeBin) {
+        const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code[u]) : -1;
+        warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code[u])), node,
+                      static_cast<uint32_t>(a.n), lane, sinks);
+        zthr = zthreshold(wb.thr, c.s, c.lse);
+      }
     }
   }
 }
 
+// Child bitmap of a CSR node in the warp's mask copy: bit c set for every
+// child code c (child ids o0 .. o1-1, codes ascending, so the rank of a code
+// among the set bits is its id minus o0). Codes are read 16 bytes at a time
+// from an 8-aligned start (the code array is padded), four loads per lane
+// in flight. Warp-collective.
+__device__ __forceinline__ void csr_bitmap(const StepArgs& a, uint32_t o0, uint32_t o1,
+                                           int words, uint32_t* wmask, int lane) {
+  for (int i = lane; i < words; i += 32) wmask[i] = 0u;
+  __syncwarp();
+  const uint32_t a0 = o0 & ~7u;
+  const uint32_t nv = (o1 - a0 + 7u) / 8u;
+  const uint4* src = reinterpret_cast<const uint4*>(a.codes + a0);
+  for (uint32_t v0 = lane; v0 < nv; v0 += 32u * 4u) {
+    uint4 q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t v = v0 + 32u * u;
+      q[u] = v < nv ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t v = v0 + 32u * u;
+      const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t id = a0 + v * 8u + e;
+        if (v < nv && id >= o0 && id < o1) {
+          const uint32_t code = (w[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
+          atomicOr(&wmask[code >> 5], 1u << (code & 31));
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // Candidate walk of a row in place in its stage (rows over 8 KB, CSR rows with
-// more children than one 32-lane batch per warp, dense rows with many
-// children).
+// more children than one 32-lane batch per warp). wmask: the warp's mask copy (room for a V-bit row).
+constexpr uint32_t kCsrBitmapMin = 192;  // CSR rows with more children use a bitmap
 template <int BF16>
 __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
                           float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
-                          const ThrSinks& sinks, int lane, int part, int nparts) {
+                          uint32_t* wmask, const ThrSinks& sinks, int lane, int part,
+                          int nparts) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   if (rmax < zthr) return;  // even the row's largest logit cannot reach the threshold
+  const uint32_t* mrow = nullptr;  // valid-child bitmap (null: every code is valid)
+  int words = 0;
   if (a.layout == SIDBEAM_LAYOUT_CSR) {
-    const uint32_t nst = csr_staged(a, c.o0, c.o1);
-    const uint32_t k_step = static_cast<uint32_t>(32 * nparts);
-    for (uint32_t k0 = c.o0 + static_cast<uint32_t>(part * 32); k0 < c.o1; k0 += k_step) {
-      const uint32_t k = k0 + lane;
-      const bool in = k < c.o1;
-      const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
-      const float z = in ? elem<BF16>(zrow, code) : 0.f;
-      const bool ok = in && z >= zthr;
-      if (!__any_sync(kFull, ok)) continue;
-      const float score = c.s + (z - c.lse);
-      warp_bin(ctl->hist, ok, score_bin(score, c.C), wb.binned, &ctl->hist_total);
-      warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(code)),
-                    static_cast<int32_t>(k), static_cast<uint32_t>(a.n), lane, sinks);
-      zthr = zthreshold(wb.thr, c.s, c.lse);
+    if (c.o1 - c.o0 <= kCsrBitmapMin) {  // all codes are staged behind the row
+      const uint32_t nst = csr_staged(a, c.o0, c.o1);
+      const uint32_t k_step = static_cast<uint32_t>(32 * nparts);
+      for (uint32_t k0 = c.o0 + static_cast<uint32_t>(part * 32); k0 < c.o1; k0 += k_step) {
+        const uint32_t k = k0 + lane;
+        const bool in = k < c.o1;
+        const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
+        const float z = in ? elem<BF16>(zrow, code) : 0.f;
+        const bool ok = in && z >= zthr;
+        if (!__any_sync(kFull, ok)) continue;
+        const float score = c.s + (z - c.lse);
+        warp_bin(ctl->hist, ok, score_bin(score, c.C), wb.binned, &ctl->hist_total);
+        warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(code)),
+                      static_cast<int32_t>(k), static_cast<uint32_t>(a.n), lane, sinks);
+        zthr = zthreshold(wb.thr, c.s, c.lse);
+      }
+      return;
     }
-    return;
+    words = (a.V + 31) / 32;
+    csr_bitmap(a, c.o0, c.o1, words, wmask, lane);
+    mrow = wmask;
+  } else if (a.layout == SIDBEAM_LAYOUT_DENSE) {
+    mrow = reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes);
+    words = a.mask_words;
   }
-  // Dense level or no trie: many children, so two passes: count every child
-  // at or above the threshold, raise the threshold from the histogram, then
-  // offer only what still reaches it.
-  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  const uint32_t* mrow = reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes);
+  // Many children: two passes. Count every child at or above the threshold,
+  // raise the threshold from the histogram, then offer only what still
+  // reaches it.
   const int nvec_all = (a.V + kPerVec - 1) / kPerVec;
   const uint4* q = reinterpret_cast<const uint4*>(zrow);
   bool have_prefix = false;
@@ -666,37 +708,42 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
     for (int v0 = part * 32; v0 < nvec_all; v0 += 32 * nparts) {
       const int v = v0 + lane;
       unsigned bits = 0u;
-      if (v < nvec_all) {
-        const uint4 x = q[v];
-        if (vec_max<BF16>(x) >= zthr) {
-          const int cb = v * kPerVec;
-          unsigned valid = (1u << kPerVec) - 1u;
-          if (dense) valid = (mrow[cb >> 5] >> (cb & 31)) & ((1u << kPerVec) - 1u);
-          for (int j = 0; j < kPerVec; ++j)
-            if (((valid >> j) & 1u) && cb + j < a.V && elem<BF16>(zrow, cb + j) >= zthr)
-              bits |= 1u << j;
-        }
+      const uint4 x = v < nvec_all ? q[v] : make_uint4(0u, 0u, 0u, 0u);
+      if (v < nvec_all && vec_max<BF16>(x) >= zthr) {
+        const int cb = v * kPerVec;
+        unsigned valid = (1u << kPerVec) - 1u;
+        if (mrow) valid = (mrow[cb >> 5] >> (cb & 31)) & ((1u << kPerVec) - 1u);
+        if (a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+#pragma unroll
+        for (int j = 0; j < kPerVec; ++j)
+          if (((valid >> j) & 1u) && vec_elem<BF16>(x, j) >= zthr) bits |= 1u << j;
+      }
+      if (pass == 0) {  // count the hits of this vector in one go
+#pragma unroll
+        for (int j = 0; j < kPerVec; ++j)
+          if ((bits >> j) & 1u)
+            atomicAdd(&ctl->hist[score_bin(c.s + (vec_elem<BF16>(x, j) - c.lse), c.C)], 1u);
+        const int cnt = static_cast<int>(__reduce_add_sync(kFull, __popc(bits)));
+        wb.binned += cnt;
+        if (lane == 0 && cnt) atomicAdd(&ctl->hist_total, static_cast<unsigned>(cnt));
+        continue;
       }
       if (!__any_sync(kFull, bits != 0u)) continue;
-      if (pass == 1 && dense && !have_prefix) {
-        dense_prefix(mrow, a.mask_words, wprefix, lane);
+      if (mrow && !have_prefix) {
+        dense_prefix(mrow, words, wprefix, lane);
         have_prefix = true;
       }
       while (__any_sync(kFull, bits != 0u)) {
         const int j = bits ? __ffs(bits) - 1 : 0;
         const int code = v * kPerVec + j;
-        const float z = bits ? elem<BF16>(zrow, code) : 0.f;
+        const float z = vec_elem<BF16>(x, j);
         const bool has = bits != 0u && z >= zthr;
         bits &= bits - 1u;
         const float score = c.s + (z - c.lse);
-        if (pass == 0) {
-          warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
-        } else {
-          const int32_t node = (has && dense) ? dense_child(mrow, wprefix, c.o0, code) : -1;
-          warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
-                        static_cast<uint32_t>(a.n), lane, sinks);
-          zthr = zthreshold(wb.thr, c.s, c.lse);
-        }
+        const int32_t node = (has && mrow) ? dense_child(mrow, wprefix, c.o0, code) : -1;
+        warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code)), node,
+                      static_cast<uint32_t>(a.n), lane, sinks);
+        zthr = zthreshold(wb.thr, c.s, c.lse);
       }
     }
     if (pass == 0) {
@@ -705,6 +752,40 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
       zthr = zthreshold(wb.thr, c.s, c.lse);
     }
   }
+}
+
+// Counts a CTA keeps before it moves them to the request's histogram.
+constexpr unsigned kPushAfter = 64;
+
+// Moves this CTA's histogram counts into request r's global histogram and
+// raises the shared bounds from the global one, which holds every CTA's
+// pushed counts (warp-collective; one warp of the CTA at a time, the others
+// skip). Counts move by atomic exchange, so each candidate stays counted
+// exactly once; the segment end pushes what is left. Only for requests split
+// over several CTAs (a CTA that holds a whole request keeps its histogram).
+__device__ void push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C, WarpBuf& wb,
+                               const ThrSinks& sinks, int lane) {
+  int got = 0;
+  if (lane == 0) got = atomicCAS(&ctl->push_lock, 0, 1) == 0 ? 1 : 0;
+  if (!__shfl_sync(kFull, got, 0)) return;
+  uint32_t* gh = a.ghist + static_cast<size_t>(r) * kHistBins;
+  for (int b = lane; b < kHistBins; b += 32) {
+    const uint32_t c = atomicExch(&ctl->hist[b], 0u);
+    if (c) atomicAdd(gh + b, c);
+  }
+  if (lane == 0) atomicExch(&ctl->hist_total, 0u);
+  __threadfence();
+  uint4 h[8];
+  const uint4* g4 = reinterpret_cast<const uint4*>(gh) + lane * 8;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) h[j] = __ldcg(g4 + j);
+  const uint64_t hb = hist_bound_regs(h, static_cast<uint32_t>(a.n), C, lane);
+  if (hb > wb.thr) {
+    wb.thr = hb;
+    publish_thr(hb, lane, sinks);
+  }
+  __syncwarp();
+  if (lane == 0) atomicExch(&ctl->push_lock, 0);
 }
 
 // Histogram reference of request r: the largest finite parent score of the
@@ -795,12 +876,8 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   int64_t lo, hi;
   a.part.range(static_cast<int>(blockIdx.x), lo, hi);
   RowSeq q;
-  if (a.coop) {
-    q = RowSeq{lo, 1, static_cast<int>(hi - lo)};
-  } else {
-    const int64_t f = lo + warp;
-    q = RowSeq{f, W, f < hi ? static_cast<int>((hi - f + W - 1) / W) : 0};
-  }
+  a.part.rows(static_cast<int>(blockIdx.x), a.coop ? 0 : warp, a.coop ? 1 : W, q.first, q.stride,
+              q.count);
   const int part = a.coop ? warp : 0;
   const int nparts = a.coop ? W : 1;
 
@@ -837,6 +914,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     ctl->ref_ord[0] = 0u;
     ctl->ref_ord[1] = 0u;
     ctl->hist_total = 0u;
+    ctl->push_lock = 0;
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
   __syncthreads();
@@ -916,14 +994,13 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     if (stopped) break;
 
     const uint32_t b = static_cast<uint32_t>(row - static_cast<int64_t>(r) * a.B_in);
+    const bool multi = a.part.contributors(r) > 1;
     RowCtx c{s, 0.f, C, b * static_cast<uint32_t>(a.V), o0, o1};
     const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
     const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
     const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
     const uint32_t nchild = o1 - o0;
-    const bool reg_row =
-        REG && (csr ? nchild <= static_cast<uint32_t>(32 * nparts)
-                    : (a.layout != SIDBEAM_LAYOUT_DENSE || nchild <= kHeavyDense * nparts));
+    const bool reg_row = REG && (!csr || nchild <= static_cast<uint32_t>(32 * nparts));
     if (reg_row) {
       uint4 x[kRegVecs];
       copy_row_regs<BF16>(zrow, a.V, lane, x);
@@ -940,10 +1017,19 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         ccode = csr_code(a, zrow, o0, csr_staged(a, o0, o1), ck);
         cz = elem<BF16>(zrow, ccode);
       }
-      ++g.consumed;
-      ring_refill(a, q, mb, g, lane, pol);  // the stage is refilled before any arithmetic
-      req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
-      req_pref_r = r;
+      // The stage goes back now at CSR levels (the walk needs nothing more from
+      // it); dense and unconstrained rows keep it until their walk is done.
+      bool held = true;
+      auto release = [&]() {
+        if (!held) return;
+        held = false;
+        __syncwarp();
+        ++g.consumed;
+        ring_refill(a, q, mb, g, lane, pol);
+        req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+        req_pref_r = r;
+      };
+      if (csr) release();
 
       const int nvec = (a.V + kPerVec - 1) / kPerVec;
       const bool full = nvec == 32 * kRegVecs && a.V % kPerVec == 0;
@@ -954,7 +1040,10 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
       float zthr = zthreshold(wb.thr, c.s, c.lse);
-      if (rmax < zthr) continue;
+      if (rmax < zthr) {
+        release();
+        continue;
+      }
       if (csr) {
         const bool ok = cin && cz >= zthr;
         if (!__any_sync(kFull, ok)) continue;
@@ -967,20 +1056,53 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         const bool any = (full && nparts == 1)
                              ? reg_hits<BF16, true>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp)
                              : reg_hits<BF16, false>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
-        if (!any) continue;
-        take_hits<BF16>(a, a.logits + row * a.row_bytes, hp, my_mask, my_prefix, c, zthr, wb,
-                        ctl, sinks, lane);
+        if (!any) {
+          release();
+          continue;
+        }
+        const int nhits = static_cast<int>(
+            __reduce_add_sync(kFull, __popc(hp[0]) + __popc(hp[1]) + __popc(hp[2]) + __popc(hp[3])));
+        if (nhits <= kOnePassHits) {
+          take_hits<BF16, kTakeBinOffer>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks,
+                                         lane);
+        } else {
+          // Many hits: count them all, raise the threshold (this CTA's histogram,
+          // then the request's), and offer only the hits that still reach it.
+          take_hits<BF16, kTakeBin>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks, lane);
+          __syncwarp();
+          refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+          if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
+            push_histogram(a, ctl, r, C, wb, sinks, lane);
+          const float zthr1 = zthreshold(wb.thr, c.s, c.lse);
+          if (zthr1 > zthr) {
+            // hits at the raised threshold: a subset of the ones counted
+#pragma unroll
+            for (int i = 0; i < kRegVecs / 4; ++i) hp[i] = 0u;
+            zthr = zthr1;
+            if (full && nparts == 1)
+              reg_hits<BF16, true>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
+            else
+              reg_hits<BF16, false>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
+          }
+          take_hits<BF16, kTakeOffer>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks,
+                                      lane);
+        }
+        release();
       }
       __syncwarp();
       refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+      if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
+        push_histogram(a, ctl, r, C, wb, sinks, lane);
     } else {
       float rmax;
       row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
       smem_walk<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
-                      sinks, lane, part, nparts);
+                      my_mask, sinks, lane, part, nparts);
       __syncwarp();
       refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+      if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
+        push_histogram(a, ctl, r, C, wb, sinks, lane);
       ++g.consumed;
       ring_refill(a, q, mb, g, lane, pol);
       req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
@@ -1050,7 +1172,7 @@ bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int
       c.off_wprefix = o;
       o += W * c.prefix_words * 4;
       c.off_wmask = o;
-      o += reg ? W * c.prefix_words * 4 : 0;
+      o += W * c.prefix_words * 4;
       o = round_up(o, 128);
       const int warp_bytes = W * cw * 12 + 256;
       const int avail = kSmemBudget - o - warp_bytes;
@@ -1139,7 +1261,10 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
 
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
   const int extra = dense ? a.mask_stride * 4 : (a.layout == SIDBEAM_LAYOUT_CSR ? 512 : 0);
-  const int prefix_words = dense ? a.mask_stride : 0;
+  // Per-warp bitmap + prefix counts: dense mask rows, and CSR nodes with many
+  // children (turned into a bitmap).
+  const int prefix_words = dense ? a.mask_stride
+                                 : (a.layout == SIDBEAM_LAYOUT_CSR ? ((V + 31) / 32 + 3) / 4 * 4 : 0);
   const bool reg = static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
   if (!choose_step_config(V, esize, extra, prefix_words, n_out, reg, &a.cfg) &&
       !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, &a.cfg)))

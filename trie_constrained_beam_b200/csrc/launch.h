@@ -25,7 +25,7 @@ struct Partition {
   int grid;
   int B_in;     // rows per request
   int maxG;     // upper bound on contributors of any request
-  int grouped;  // 1: request r owns CTAs r*G .. r*G+G-1
+  int grouped;  // 1: request r owns CTAs r*G .. r*G+G-1 (its slots interleaved)
   int G;
 
   __host__ __device__ __forceinline__ void range(int cta, int64_t& lo, int64_t& hi) const {
@@ -40,6 +40,31 @@ struct Partition {
       hi = lo + rows_per_cta;
       if (hi > total_rows) hi = total_rows;
     }
+  }
+  // The rows of a CTA as a strided sequence first + stride * i, i < count. A
+  // request's group of CTAs interleaves its parent slots (CTA j takes slots
+  // j, j+G, j+2G, ...), so that every CTA gets its share of the best parents
+  // (the beam is ranked best-first) and the candidate work stays balanced.
+  // `part` of `parts` (warps dealt rows round-robin) narrows it to one warp's
+  // rows; parts = 1 gives the whole CTA's sequence.
+  __host__ __device__ __forceinline__ void rows(int cta, int part, int parts, int64_t& first,
+                                                int64_t& stride, int& count) const {
+    int64_t f, st, n;
+    if (grouped) {
+      const int r = cta / G, j = cta - r * G;
+      f = static_cast<int64_t>(r) * B_in + j;
+      st = G;
+      n = (B_in - j + G - 1) / G;
+    } else {
+      int64_t lo, hi;
+      range(cta, lo, hi);
+      f = lo;
+      st = 1;
+      n = hi - lo;
+    }
+    first = f + st * part;
+    stride = st * parts;
+    count = part < n ? static_cast<int>((n - part + parts - 1) / parts) : 0;
   }
   __host__ __device__ __forceinline__ int first_cta(int r) const {
     if (grouped) return r * G;

@@ -238,6 +238,42 @@ __device__ __forceinline__ uint64_t hist_bound(const uint32_t* hist, uint32_t n,
   return key_floor(C - static_cast<float>(k + 2) / kHistScale);
 }
 
+// hist_bound over a histogram held in registers: lane l holds bins 32l .. 32l+31
+// as h[0..7] (four bins each, in order).
+__device__ __forceinline__ uint64_t hist_bound_regs(const uint4 (&h)[8], uint32_t n, float C,
+                                                    int lane) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s += h[j].x + h[j].y + h[j].z + h[j].w;
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned b = __ballot_sync(0xFFFFFFFFu, incl >= n);
+  if (b == 0) return 0ull;
+  const int src = __ffs(b) - 1;
+  int k = 0;
+  if (lane == src) {
+    uint32_t cum = incl - s;
+    int found = -1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t v[4] = {h[j].x, h[j].y, h[j].z, h[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cum += v[e];
+        if (found < 0 && cum >= n) found = 4 * j + e;
+      }
+    }
+    k = lane * 32 + found;
+  }
+  k = __shfl_sync(0xFFFFFFFFu, k, src);
+  if (k >= kHistBins - 2) return 0ull;
+  return key_floor(C - static_cast<float>(k + 2) / kHistScale);
+}
+
 // ------------------------------------------------------------ shared control
 struct SelCtl {
   unsigned long long cta_thr;  // CTA-wide lower bound on the segment's n-th best key
@@ -251,7 +287,8 @@ struct SelCtl {
   int abort_flag;
   int staged;
   int rank_bad;                // rank merge: the entries did not match the histogram
-  unsigned hist_total;         // candidates counted in `hist` this segment
+  unsigned hist_total;         // candidates counted in `hist` and not yet pushed
+  int push_lock;               // beam_step: one warp at a time moves `hist` to the request's
   unsigned ref_ord[2];         // beam_step: max parent score (ordered) of a segment, by parity
   int wcount[32];
   int segoff[kMaxSegCounts + 1];
