@@ -268,6 +268,10 @@ def run_ours(args, world, rank, local):
         e2e = {"value": world * K2 * logits_per_search / (ems * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K2}
 
+    cat_lines = None
+    if not args.no_catalog:
+        cat_lines = measure_catalog(tcb, trie, cat, w, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds, cat=cat)
@@ -289,11 +293,53 @@ def run_ours(args, world, rank, local):
                   "3 rotating logits copies; per-step times from events inside the graph",
         "logits_per_step": logits_per_search,
         "e2e": e2e,
+        "catalog_score": cat_lines,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": K * (w.depth + 1),
     }
     return line
+
+
+def measure_catalog(tcb, trie4, cat4, w4, dev):
+    """catalog_score_topk throughput ((request, SID) pairs scored per second):
+    the SPRINT-like workload (32 requests, 50,000 SIDs, 4 x 256, top-10) and the
+    wide-beam catalog (8M SIDs, 5 x 4096) with 32 requests, top-10. Tables are
+    seeded per-position log-softmax tables, resident in HBM."""
+    import torch
+    from sidgen import host
+    from sidgen.workloads import WORKLOADS
+
+    def run(trie, n_leaves, R, L, V, K, seed, sigma, reps=50):
+        table = torch.from_numpy(host.table_logits(seed, R, L, V, sigma)).to(dev).log_softmax(-1)
+        table = table.contiguous()
+        out_s = torch.empty((R, K), device=dev)
+        out_l = torch.empty((R, K), dtype=torch.int32, device=dev)
+        ws = torch.zeros(tcb.catalog_score_workspace_size(trie, R, K), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            tcb.catalog_score_topk(trie, table, R, K, out_s, out_l, ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            tcb.catalog_score_topk(trie, table, R, K, out_s, out_l, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        assert tcb.sidbeam_get_device_status(ws) == 0
+        return {"us_per_call": us, "pairs_per_s": R * n_leaves / (us * 1e-6),
+                "requests": R, "sids": n_leaves, "depth": L, "codes_per_level": V, "K": K}
+
+    w2 = WORKLOADS[2]
+    cat2 = w2.catalog()
+    trie2 = tcb.sid_trie_build(cat2, w2.codes_per_level, w2.layouts)
+    a = run(trie2, _n_leaves(cat2), w2.R, w2.depth, w2.V, w2.K, w2.logits_seed, w2.table_sigma)
+    b = run(trie4, _n_leaves(cat4), 32, w4.depth, w4.V, 10, w4.logits_seed + 7, 1.5, reps=10)
+    return {"unit": "(request, SID) pairs/s", "sprint_opq_50k": a, "wide_beam_8M_x32": b}
+
+
+def _n_leaves(cat):
+    return int(np.asarray(cat).shape[0])  # the recipes draw distinct SIDs
 
 
 def _profile_traffic():
@@ -428,6 +474,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-catalog", action="store_true",
+                    help="skip the catalog_score_topk throughput lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--copies", type=int, default=COPIES,
                     help="rotating copies of the per-step logits (3 keeps reads out of L2)")

@@ -48,6 +48,9 @@ constexpr int kRegVecs = 16;  // 16-byte vectors per lane held in registers (8 K
 // A register row with more hits than this is walked in two passes (count,
 // raise the threshold, offer).
 constexpr int kOnePassHits = 64;
+// Dense rows with more children than this are walked in place in their stage
+// (counting there goes a vector at a time).
+constexpr uint32_t kHugeDense = 2048;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 // f(I) for I = 0 .. N-1 with I a compile-time constant (keeps register arrays
@@ -661,7 +664,8 @@ __device__ __forceinline__ void csr_bitmap(const StepArgs& a, uint32_t o0, uint3
 }
 
 // Candidate walk of a row in place in its stage (rows over 8 KB, CSR rows with
-// more children than one 32-lane batch per warp). wmask: the warp's mask copy (room for a V-bit row).
+// more children than one 32-lane batch per warp, dense rows with very many
+// children). wmask: the warp's mask copy (room for a V-bit row).
 constexpr uint32_t kCsrBitmapMin = 192;  // CSR rows with more children use a bitmap
 template <int BF16>
 __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
@@ -1000,7 +1004,8 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
     const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
     const uint32_t nchild = o1 - o0;
-    const bool reg_row = REG && (!csr || nchild <= static_cast<uint32_t>(32 * nparts));
+    const bool reg_row = REG && (csr ? nchild <= static_cast<uint32_t>(32 * nparts)
+                                     : (a.layout != SIDBEAM_LAYOUT_DENSE || nchild <= kHugeDense));
     if (reg_row) {
       uint4 x[kRegVecs];
       copy_row_regs<BF16>(zrow, a.V, lane, x);
