@@ -215,6 +215,21 @@ int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K
                        float* out_scores, int32_t* out_leaf, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- SID-range lm_head
+ * lmhead_logits -- flashrec 0.1.0, Features > Decoding ("SID constraint"): the
+ * lm_head evaluated only over the SID token range. For every row and code:
+ *   logits[row][c] = sum_k hidden[row][k] * w_sid[c][k]
+ * with bf16 inputs (exact products) and fp32 accumulation on the tensor cores
+ * (tcgen05; the summation order is not specified).
+ *  hidden     device bf16 [M][d], row-major, 16-byte aligned; d % 8 == 0.
+ *  w_sid      device bf16 [V][d], row-major, 16-byte aligned (the rows of the
+ *             lm_head weight that belong to the level's SID codes).
+ *  logits     device f32 [M][ld], ld >= V, ld % 4 == 0, 16-byte aligned.
+ *  workspace  device, >= 256 bytes, zero-filled before first use (status word).
+ * Asynchronous on `stream`. Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA. */
+int lmhead_logits(const void* hidden, const void* w_sid, int M, int V, int d, float* logits,
+                  int64_t ld, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- status
  * sidbeam_get_device_status -- synchronises `stream`, reads and clears the
  * status word that beam_step / catalog_score_topk keep at the start of

@@ -41,7 +41,7 @@ EXPORTED = (
     "sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
     "sid_trie_free", "beam_step_workspace_size", "beam_step", "beam_finalize",
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
-    "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc",
+    "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc", "lmhead_logits",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -81,13 +81,14 @@ def load():
     L.catalog_score_workspace_size.restype = SZ
     L.catalog_score_topk.argtypes = [P, P, I32, I32, P, P, P, SZ, P]
     L.sidbeam_get_device_status.argtypes = [P, P]
+    L.lmhead_logits.argtypes = [P, P, I32, I32, I32, P, I64, P, SZ, P]
     L.sidbeam_last_error.argtypes = []
     L.sidbeam_last_error.restype = ctypes.c_char_p
     L.sidbeam_version.argtypes = []
     L.sidbeam_version.restype = ctypes.c_char_p
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
                  "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
-                 "sidbeam_get_device_status"):
+                 "sidbeam_get_device_status", "lmhead_logits"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -233,6 +234,16 @@ def catalog_score_topk(trie, logp, R, K, out_scores, out_leaf, workspace, stream
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check(rc)
+
+
+def lmhead_logits(hidden, w_sid, out, workspace, stream=None):
+    """out[row][c] = sum_k hidden[row][k] * w_sid[c][k] (bf16 in, fp32 out) on the
+    tensor cores. hidden [M][d], w_sid [V][d] bf16; out f32 [M][>= V]."""
+    M, d = hidden.shape
+    V = w_sid.shape[0]
+    _check(load().lmhead_logits(_ptr(hidden), _ptr(w_sid), M, V, d, _ptr(out), out.stride(0),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)))
 
 
 def sidbeam_get_device_status(workspace, stream=None) -> int:
