@@ -230,6 +230,26 @@ int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K
 int lmhead_logits(const void* hidden, const void* w_sid, int M, int V, int d, float* logits,
                   int64_t ld, void* workspace, size_t workspace_bytes, void* stream);
 
+/* sidbeam_fused_lmhead_step -- flashrec 0.1.0, Features > Decoding ("SID
+ * constraint"): the lm_head over the SID token range feeding the constrained
+ * step, without writing the logits out. Computes exactly beam_step's result
+ * for logits[row][c] = sum_k hidden[row][k] * w_sid[c][k] (fp32 accumulation
+ * on the tensor cores, as lmhead_logits):
+ *  hidden          device bf16 [R*B_in][d], row-major, 16-byte aligned, d % 8 == 0.
+ *  w_sid           device bf16 [V][d], row-major, 16-byte aligned.
+ *  every other argument as for beam_step (no dtype / ld: the logits are made
+ *  here); workspace >= fused_lmhead_workspace_size(R, B_in, n_out, V) bytes,
+ *  zero-filled before first use (the call leaves the first part zeroed; the
+ *  rest is scratch: per-row child bitmaps, per-tile partial sums, child logits).
+ * Asynchronous on `stream` (three launches). Errors as for beam_step. */
+size_t fused_lmhead_workspace_size(int R, int B_in, int n_out, int V);
+int sidbeam_fused_lmhead_step(const sidbeam_trie* trie, int step, const void* hidden,
+                              const void* w_sid, int d, const float* parent_scores,
+                              const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                              float* out_scores, int32_t* out_parent, int32_t* out_code,
+                              int32_t* out_node, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* ---------------------------------------------------------------- status
  * sidbeam_get_device_status -- synchronises `stream`, reads and clears the
  * status word that beam_step / catalog_score_topk keep at the start of

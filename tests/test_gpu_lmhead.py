@@ -91,3 +91,86 @@ def test_lmhead_logits_argument_checks(tcb):
     with pytest.raises(native.SidbeamError) as e:
         tcb.lmhead_logits(h, wt, out, ws)
     assert e.value.status == native.SIDBEAM_ERR_ALIGNMENT
+
+
+# ------------------------------------------------------------------ fused step
+def _fused_case(tcb, trie_o, trie_g, step, R, B_in, n, V, d, seed, level_nodes, w_sigma=0.05):
+    """One fused step on seeded inputs; parents are distinct level-`step` nodes
+    with scores ranked best-first. Returns GPU outputs and the oracle inputs."""
+    import torch
+    from trie_constrained_beam_b200 import native
+    rng = np.random.default_rng(seed)
+    M = R * B_in
+    if step == 0:
+        pn = np.zeros(M, dtype=np.int32)
+        ps = np.zeros(M, dtype=np.float32)
+    else:
+        pn = np.concatenate([rng.choice(level_nodes, size=B_in, replace=False)
+                             for _ in range(R)]).astype(np.int32)
+        ps = np.concatenate([np.sort(rng.uniform(-12, -2, size=B_in))[::-1]
+                             for _ in range(R)]).astype(np.float32)
+        ps[rng.random(M) < 0.05] = -np.inf          # a few dead rows
+    hb = host.f32_to_bf16_bits(rng.standard_normal((M, d)).astype(np.float32))
+    wb = host.f32_to_bf16_bits((w_sigma * rng.standard_normal((V, d))).astype(np.float32))
+    dev = "cuda"
+    out_s = torch.empty(R * n, dtype=torch.float32, device=dev)
+    out_p, out_c, out_n = (torch.empty(R * n, dtype=torch.int32, device=dev) for _ in range(3))
+    ws = torch.zeros(tcb.fused_lmhead_workspace_size(R, B_in, n, V), dtype=torch.uint8, device=dev)
+    tcb.fused_lmhead_step(trie_g, step, _dev_bf16(hb), _dev_bf16(wb),
+                          torch.from_numpy(ps).to(dev), torch.from_numpy(pn).to(dev),
+                          R, B_in, n, out_s, out_p, out_c, out_n, ws)
+    assert tcb.sidbeam_get_device_status(ws) == 0
+    gpu = {"score": out_s.view(R, n).cpu().numpy(), "parent": out_p.view(R, n).cpu().numpy(),
+           "code": out_c.view(R, n).cpu().numpy(), "node": out_n.view(R, n).cpu().numpy()}
+    return gpu, hb, wb, ps, pn
+
+
+def _fused_tol(tcb, hb, wb, rows):
+    """Score tolerance of the fused step: the step's own TOL plus twice the
+    largest error of the tensor-core logits on these rows against the exact
+    dot products (a score is s + z - lse; neither z nor lse moves by more
+    than the largest logit error)."""
+    from parity import TOL
+    got = _run(tcb, hb[rows], wb)[:, :wb.shape[0]]
+    dz = float(np.abs(got - oracle.lmhead_logits(hb[rows], wb)).max())
+    return TOL + 2.0 * dz
+
+
+@pytest.mark.parametrize("layouts", [[1, 1, 1], [2, 2, 2], [1, 2, 2], None])
+def test_fused_step_small_matches_oracle(tcb, layouts):
+    """Steps 0-2 of a 3-level, V=512 catalog, every layout and no trie, d = 136
+    (a K tail); ranks compared with the tie-aware rule."""
+    from parity import compare_step
+    V, d, R, B_in, n = 512, 136, 3, 24, 16
+    cat = host.draw_catalog(31, 3000, [V] * 3)
+    to = oracle.OracleTrie(cat, [V] * 3)
+    tg = tcb.sid_trie_build(cat, [V] * 3, layouts) if layouts is not None else None
+    for step in range(3):
+        Bi = 1 if step == 0 else B_in
+        nodes = np.arange(to.n_nodes(step))
+        if step > 0 and nodes.size < Bi:
+            continue
+        gpu, hb, wb, ps, pn = _fused_case(tcb, to, tg, step, R, Bi, n, V, d, 700 + step, nodes)
+        z = oracle.lmhead_logits(hb, wb)
+        compare_step(gpu, to if tg is not None else None, step, z, ps, pn, R, Bi, n, V,
+                     tol=_fused_tol(tcb, hb, wb, slice(None)))
+
+
+def test_fused_step_full_size_sampled_requests(tcb):
+    """The fused-lm_head workload at full size (32 x 128 rows, V = 8192,
+    d = 2048, W ~ N(0, 0.02), 1M-SID catalog): step 1 on the GPU for every
+    request; two requests compared against the oracle."""
+    from parity import compare_step
+    w = WORKLOADS[5]
+    cat = w.catalog()
+    to = oracle.OracleTrie(cat, w.codes_per_level)
+    tg = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    nodes = np.arange(to.n_nodes(1))
+    gpu, hb, wb, ps, pn = _fused_case(tcb, to, tg, 1, w.R, w.n, w.n, w.V, w.hidden_dim, 55, nodes,
+                                      w_sigma=w.weight_sigma)
+    for r in (0, w.R - 1):
+        rows = slice(r * w.n, (r + 1) * w.n)
+        z = oracle.lmhead_logits(hb[rows], wb)
+        sub = {k: v[r:r + 1] for k, v in gpu.items()}
+        compare_step(sub, to, 1, z, ps[rows], pn[rows], 1, w.n, w.n, w.V,
+                     tol=_fused_tol(tcb, hb, wb, rows))

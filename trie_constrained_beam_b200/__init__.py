@@ -13,6 +13,8 @@ from .native import (  # noqa: F401
     beam_step_workspace_size,
     catalog_score_topk,
     catalog_score_workspace_size,
+    fused_lmhead_step,
+    fused_lmhead_workspace_size,
     lmhead_logits,
     sid_trie_build,
     sid_trie_info,

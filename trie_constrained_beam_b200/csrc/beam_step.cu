@@ -235,15 +235,6 @@ __device__ __forceinline__ void row_stats(const uint8_t* row, int V, int lane, f
   lse_out = m + logf(sum);
 }
 
-// Lowest logit a child needs to reach the key threshold `thr`, loosened by a
-// relative margin far above fp32 rounding: z < zthr implies key < thr, so
-// skipping such codes never drops a candidate the exact key test would keep.
-__device__ __forceinline__ float zthreshold(uint64_t thr, float s, float lse) {
-  if (thr == 0ull) return __int_as_float(0xFF800000);
-  const float T = key_score(thr);
-  const float margin = 1e-4f * (1.f + fabsf(T) + fabsf(s) + fabsf(lse));
-  return ((T - s) + lse) - margin;
-}
 
 // --------------------------------------------------------------- register rows
 // Element j of a 16-byte vector (8 bf16 or 4 fp32), j warp-divergent.

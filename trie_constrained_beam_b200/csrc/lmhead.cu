@@ -418,3 +418,59 @@ extern "C" int lmhead_logits(const void* hidden, const void* w_sid, int M, int V
   a.status = static_cast<uint32_t*>(workspace);
   return launch_lmhead_gemm(hidden, w_sid, a, static_cast<cudaStream_t>(stream));
 }
+
+namespace sidbeam {
+int launch_fused_lmhead(const sidbeam_trie* trie, int step, const void* hidden,
+                        const void* w_sid, int d, const float* parent_scores,
+                        const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                        float* out_scores, int32_t* out_parent, int32_t* out_code,
+                        int32_t* out_node, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+size_t fused_lmhead_workspace(int R, int B_in, int n_out, int V);
+}  // namespace sidbeam
+
+extern "C" size_t fused_lmhead_workspace_size(int R, int B_in, int n_out, int V) {
+  if (R < 1 || B_in < 1 || n_out < 1 || n_out > SIDBEAM_MAX_BEAM || V < 1 || V > SIDBEAM_MAX_V)
+    return 0;
+  return fused_lmhead_workspace(R, B_in, n_out, V);
+}
+
+extern "C" int sidbeam_fused_lmhead_step(const sidbeam_trie* trie, int step, const void* hidden,
+                                         const void* w_sid, int d, const float* parent_scores,
+                                         const int32_t* parent_nodes, int R, int B_in, int n_out,
+                                         int V, float* out_scores, int32_t* out_parent,
+                                         int32_t* out_code, int32_t* out_node, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (!hidden || !w_sid || !parent_scores || !out_scores || !out_parent || !out_code || !out_node)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: NULL pointer argument");
+  if (trie && !parent_nodes)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: parent_nodes is NULL with a trie");
+  if (R < 1 || B_in < 1 || d < 1)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: R=%d B_in=%d d=%d", R, B_in, d);
+  if (n_out < 1 || n_out > SIDBEAM_MAX_BEAM)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: n_out=%d outside [1, %d]", n_out,
+                     SIDBEAM_MAX_BEAM);
+  if (V < 1 || V > SIDBEAM_MAX_V)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: V=%d unsupported", V);
+  if (static_cast<uint64_t>(B_in) * static_cast<uint64_t>(V) > 0xFFFFFFFFull ||
+      static_cast<int64_t>(R) * B_in > 0x7FFFFFFFll || static_cast<int64_t>(R) * n_out > 0x7FFFFFFFll)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: shape too large");
+  if ((d & 7) != 0 || (reinterpret_cast<uintptr_t>(hidden) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(w_sid) & 15u) != 0)
+    return set_error(SIDBEAM_ERR_ALIGNMENT,
+                     "fused_lmhead_step: hidden and w_sid 16-byte aligned, d %% 8 == 0");
+  if (trie) {
+    if (step < 0 || step >= trie->depth)
+      return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: step %d outside [0, %d)", step,
+                       trie->depth);
+    if (trie->V[step] != V)
+      return set_error(SIDBEAM_ERR_INVALID_ARG,
+                       "fused_lmhead_step: V=%d but the trie has V=%d at level %d", V,
+                       trie->V[step], step + 1);
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return set_error(SIDBEAM_ERR_WORKSPACE, "fused_lmhead_step: workspace must be 256-byte aligned");
+  return launch_fused_lmhead(trie, step, hidden, w_sid, d, parent_scores, parent_nodes, R, B_in,
+                             n_out, V, out_scores, out_parent, out_code, out_node, workspace,
+                             workspace_bytes, static_cast<cudaStream_t>(stream));
+}

@@ -274,6 +274,16 @@ __device__ __forceinline__ uint64_t hist_bound_regs(const uint4 (&h)[8], uint32_
   return key_floor(C - static_cast<float>(k + 2) / kHistScale);
 }
 
+// Lowest logit a child needs to reach the key threshold `thr`, loosened by a
+// relative margin far above fp32 rounding: z < zthr implies key < thr, so
+// skipping such codes never drops a candidate the exact key test would keep.
+__device__ __forceinline__ float zthreshold(uint64_t thr, float s, float lse) {
+  if (thr == 0ull) return __int_as_float(0xFF800000);
+  const float T = key_score(thr);
+  const float margin = 1e-4f * (1.f + fabsf(T) + fabsf(s) + fabsf(lse));
+  return ((T - s) + lse) - margin;
+}
+
 // ------------------------------------------------------------ shared control
 struct SelCtl {
   unsigned long long cta_thr;  // CTA-wide lower bound on the segment's n-th best key

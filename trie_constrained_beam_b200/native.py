@@ -42,6 +42,7 @@ EXPORTED = (
     "sid_trie_free", "beam_step_workspace_size", "beam_step", "beam_finalize",
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
     "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc", "lmhead_logits",
+    "fused_lmhead_workspace_size", "sidbeam_fused_lmhead_step",
 )
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -82,13 +83,17 @@ def load():
     L.catalog_score_topk.argtypes = [P, P, I32, I32, P, P, P, SZ, P]
     L.sidbeam_get_device_status.argtypes = [P, P]
     L.lmhead_logits.argtypes = [P, P, I32, I32, I32, P, I64, P, SZ, P]
+    L.fused_lmhead_workspace_size.argtypes = [I32, I32, I32, I32]
+    L.fused_lmhead_workspace_size.restype = SZ
+    L.sidbeam_fused_lmhead_step.argtypes = [P, I32, P, P, I32, P, P, I32, I32, I32, I32, P, P, P,
+                                            P, P, SZ, P]
     L.sidbeam_last_error.argtypes = []
     L.sidbeam_last_error.restype = ctypes.c_char_p
     L.sidbeam_version.argtypes = []
     L.sidbeam_version.restype = ctypes.c_char_p
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
                  "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
-                 "sidbeam_get_device_status", "lmhead_logits"):
+                 "sidbeam_get_device_status", "lmhead_logits", "sidbeam_fused_lmhead_step"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -244,6 +249,24 @@ def lmhead_logits(hidden, w_sid, out, workspace, stream=None):
     _check(load().lmhead_logits(_ptr(hidden), _ptr(w_sid), M, V, d, _ptr(out), out.stride(0),
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)))
+
+
+def fused_lmhead_workspace_size(R: int, B_in: int, n_out: int, V: int) -> int:
+    return int(load().fused_lmhead_workspace_size(R, B_in, n_out, V))
+
+
+def fused_lmhead_step(trie, step, hidden, w_sid, parent_scores, parent_nodes, R, B_in, n_out,
+                      out_scores, out_parent, out_code, out_node, workspace, stream=None):
+    """beam_step on logits = hidden @ w_sid.T made on the tensor cores and never
+    written out. hidden bf16 [R*B_in][d], w_sid bf16 [V][d]."""
+    d = hidden.shape[1]
+    V = w_sid.shape[0]
+    rc = load().sidbeam_fused_lmhead_step(
+        None if trie is None else trie.handle, step, _ptr(hidden), _ptr(w_sid), d,
+        _ptr(parent_scores), _ptr(parent_nodes), R, B_in, n_out, V, _ptr(out_scores),
+        _ptr(out_parent), _ptr(out_code), _ptr(out_node), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
 
 
 def sidbeam_get_device_status(workspace, stream=None) -> int:
