@@ -271,6 +271,9 @@ def run_ours(args, world, rank, local):
     cat_lines = None
     if not args.no_catalog:
         cat_lines = measure_catalog(tcb, trie, cat, w, dev)
+    fused = None
+    if not args.no_fused:
+        fused = measure_fused(tcb, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -294,6 +297,7 @@ def run_ours(args, world, rank, local):
         "logits_per_step": logits_per_search,
         "e2e": e2e,
         "catalog_score": cat_lines,
+        "fused_lmhead": fused,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": K * (w.depth + 1),
@@ -336,6 +340,61 @@ def measure_catalog(tcb, trie4, cat4, w4, dev):
     a = run(trie2, _n_leaves(cat2), w2.R, w2.depth, w2.V, w2.K, w2.logits_seed, w2.table_sigma)
     b = run(trie4, _n_leaves(cat4), 32, w4.depth, w4.V, 10, w4.logits_seed + 7, 1.5, reps=10)
     return {"unit": "(request, SID) pairs/s", "sprint_opq_50k": a, "wide_beam_8M_x32": b}
+
+
+def measure_fused(tcb, dev, reps=20):
+    """The fused lm_head workload (32 requests x beam 128 = 4,096 rows, d = 2,048,
+    V = 8,192, 1M-SID catalog): the tcgen05 GEMM alone (fp32 logits written) and
+    the whole fused step 1 (child bitmaps + GEMM with the lse/child epilogue +
+    selection; logits never written). Seeded inputs resident in HBM."""
+    import torch
+    from sidgen import host
+    from sidgen.workloads import WORKLOADS
+
+    w = WORKLOADS[5]
+    M, V, d, R, B_in, n = w.R * w.n, w.V, w.hidden_dim, w.R, w.n, w.n
+    rng = np.random.default_rng(5005)
+    hashes = rng.integers(0, 2 ** 63, size=M, dtype=np.int64).view(np.uint64)
+    h = torch.from_numpy(host.hidden_states(w.logits_seed, hashes, d, w.hidden_sigma)
+                         .view(np.int16)).to(dev).view(torch.bfloat16)
+    wt = torch.from_numpy(host.weight_matrix(w.weight_seed, V, d, w.weight_sigma)
+                          .view(np.int16)).to(dev).view(torch.bfloat16)
+    cat = w.catalog()
+    trie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    n1 = int(tcb.sid_trie_info(trie, 1)[0])
+    pn = torch.from_numpy(np.concatenate([rng.choice(n1, size=B_in, replace=False)
+                                          for _ in range(R)]).astype(np.int32)).to(dev)
+    ps = torch.from_numpy(np.concatenate([np.sort(rng.uniform(-12, -2, size=B_in))[::-1]
+                                          for _ in range(R)]).astype(np.float32)).to(dev)
+    logits = torch.empty((M, V), dtype=torch.float32, device=dev)
+    ws0 = torch.zeros(256, dtype=torch.uint8, device=dev)
+    outs = [torch.empty(R * n, dtype=torch.float32, device=dev)] + \
+        [torch.empty(R * n, dtype=torch.int32, device=dev) for _ in range(3)]
+    ws = torch.zeros(tcb.fused_lmhead_workspace_size(R, B_in, n, V), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    us_gemm = timed(lambda: tcb.lmhead_logits(h, wt, logits, ws0))
+    us_step = timed(lambda: tcb.fused_lmhead_step(trie, 1, h, wt, ps, pn, R, B_in, n, *outs, ws))
+    assert tcb.sidbeam_get_device_status(ws) == 0 and tcb.sidbeam_get_device_status(ws0) == 0
+    flops = 2.0 * M * V * d
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak = float(json.load(open(pk))["bf16_tflops"]) if os.path.exists(pk) else 1590.0
+    return {"rows": M, "V": V, "d": d, "gflop_per_step": flops / 1e9,
+            "gemm_us": us_gemm, "gemm_tflops": flops / (us_gemm * 1e-6) / 1e12,
+            "gemm_frac_of_bf16_peak": flops / (us_gemm * 1e-6) / 1e12 / peak,
+            "bf16_peak_tflops": peak, "fused_step_us": us_step,
+            "fused_step_tflops": flops / (us_step * 1e-6) / 1e12}
 
 
 def _n_leaves(cat):
@@ -474,6 +533,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the fused lm_head (tcgen05) lines")
     ap.add_argument("--no-catalog", action="store_true",
                     help="skip the catalog_score_topk throughput lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

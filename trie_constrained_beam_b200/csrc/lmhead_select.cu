@@ -36,6 +36,7 @@ using namespace dev;
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr int kSelWarps = 8;
+constexpr int kBatch = 16;  // child logits loaded per lane per round
 constexpr float kL2e = 1.4426950408889634f;
 
 struct FusedLayout {
@@ -317,15 +318,16 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
       }
       before = pre + incl - mine;
     }
-    // Walk the lane's set bits four at a time (independent logit loads).
+    // Walk the lane's set bits kBatch at a time (independent logit loads in
+    // flight together; a node may have thousands of children).
     int cw = l0;
     uint32_t bits = cw < l1 ? word(cw) : 0u;
     float zthr = zthreshold(wb.thr, s, lse);
     while (true) {
-      int code[4];
-      int32_t node[4];
+      int code[kBatch];
+      int32_t node[kBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kBatch; ++u) {
         while (bits == 0u && cw < l1) {
           before += __popc(word(cw));
           ++cw;
@@ -344,12 +346,12 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
         }
       }
       if (!__any_sync(kFull, code[0] >= 0)) break;
-      float z[4];
+      float z[kBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < kBatch; ++u)
         z[u] = code[u] >= 0 ? __ldcg(a.zlog + row * a.V + code[u]) : 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kBatch; ++u) {
         const bool has = code[u] >= 0 && z[u] >= zthr;
         if (!__any_sync(kFull, has)) continue;
         const float score = s + (z[u] - lse);
