@@ -37,6 +37,8 @@ using namespace dev;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr int kSelWarps = 8;
 constexpr int kBatch = 16;  // child logits loaded per lane per round
+constexpr uint32_t kHeavyChildren = 1024;  // parents with more children are walked by the CTA
+constexpr int kHeavyList = 64;             // deferred parents per segment (more: walked at once)
 constexpr float kL2e = 1.4426950408889634f;
 
 struct FusedLayout {
@@ -186,6 +188,9 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
   p += 1024;
   uint32_t* whist = reinterpret_cast<uint32_t*>(p);     // 2 x 1024 words (>= W x 256)
   p += 8192;
+  int64_t* heavy = reinterpret_cast<int64_t*>(p);        // deferred rows of the segment
+  int* heavy_count = reinterpret_cast<int*>(heavy + kHeavyList);
+  p += kHeavyList * 8 + 128;
   uint64_t* wkeys = reinterpret_cast<uint64_t*>(p);
   p += static_cast<size_t>(kSelWarps) * a.Cw * 8;
   int32_t* wvals = reinterpret_cast<int32_t*>(p);
@@ -201,6 +206,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
     ctl->hist_total = 0u;
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
+  if (threadIdx.x == 0) *heavy_count = 0;
   __syncthreads();
 
   int64_t seq_first, seq_stride;
@@ -221,51 +227,12 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
   const SelWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
                          static_cast<uint32_t>(a.V)};
   int cur_r = r_first;
-  auto flush = [&]() -> bool {
-    FlushArgs f;
-    f.n = a.n;
-    f.r = cur_r;
-    f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
-    f.G = a.part.contributors(cur_r);
-    f.maxG = a.part.maxG;
-    f.pcap = partial_cap(a.n);
-    f.part_keys = a.part_keys;
-    f.part_vals = a.part_vals;
-    f.part_count = a.part_count;
-    f.tickets = a.tickets;
-    f.request_thr = a.request_thr;
-    f.ghist = a.ghist;
-    f.C = C;
-    f.wkeys = wkeys;
-    f.cw = a.Cw;
-    f.sort_keys = wkeys;
-    f.sort_vals = wvals;
-    f.sort_cap = kSelWarps * a.Cw;
-    f.radix_hist = cta_hist;
-    f.wvals = wvals;
-    f.rank_P = whist;
-    f.rank_cur = whist + kHistBins;
-    f.direct_keys = nullptr;
-    f.direct_vals = nullptr;
-    f.direct_cap = 0;
-    const bool stop = segment_flush(team, wb, ctl, f, writer);
-    wb.count = 0;
-    wb.thr = 0ull;
-    if (stop) return true;
-    if (cur_r < r_last) C = request_reference(a, team, ctl, cur_r + 1, ref_slot ^= 1);
-    ++cur_r;
-    return false;
-  };
-
-  bool stopped = false;
-  for (int i = 0; i < seq_count && !stopped; ++i) {
-    const int64_t row = seq_first + seq_stride * i;
-    const int r = static_cast<int>(row / a.B_in);
-    while (r > cur_r && !stopped) stopped = flush();
-    if (stopped) break;
+  // Scores row `row` (of request r): this warp takes part `part` of `nparts`
+  // of the row's bitmap words.
+  auto do_row = [&](int64_t row, int r, int part, int nparts) {
     const float s = a.parent_scores[row];
     const int32_t pn = a.layout ? a.parent_nodes[row] : 0;
-    if (s == __int_as_float(0xFF800000) || pn < 0) continue;  // dead row (bad nodes: bitmap 0)
+    if (s == __int_as_float(0xFF800000) || pn < 0) return;  // dead row (bad nodes: bitmap 0)
     // lse from the per-tile partials (over all V codes of the level).
     float mj = __int_as_float(0xFF800000);
     for (int t = lane; t < a.ntiles; t += 32) mj = fmaxf(mj, a.partial[row * a.ntiles + t].x);
@@ -363,6 +330,71 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
     }
     __syncwarp();
     refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+  };
+
+  auto flush = [&]() -> bool {
+    team_sync(team);
+    const int nh = min(*reinterpret_cast<volatile int*>(heavy_count), kHeavyList);
+    for (int h = 0; h < nh; ++h) do_row(heavy[h], cur_r, warp, kSelWarps);
+    team_sync(team);
+    if (team.tid == 0) *heavy_count = 0;
+    FlushArgs f;
+    f.n = a.n;
+    f.r = cur_r;
+    f.k = static_cast<int>(blockIdx.x) - a.part.first_cta(cur_r);
+    f.G = a.part.contributors(cur_r);
+    f.maxG = a.part.maxG;
+    f.pcap = partial_cap(a.n);
+    f.part_keys = a.part_keys;
+    f.part_vals = a.part_vals;
+    f.part_count = a.part_count;
+    f.tickets = a.tickets;
+    f.request_thr = a.request_thr;
+    f.ghist = a.ghist;
+    f.C = C;
+    f.wkeys = wkeys;
+    f.cw = a.Cw;
+    f.sort_keys = wkeys;
+    f.sort_vals = wvals;
+    f.sort_cap = kSelWarps * a.Cw;
+    f.radix_hist = cta_hist;
+    f.wvals = wvals;
+    f.rank_P = whist;
+    f.rank_cur = whist + kHistBins;
+    f.direct_keys = nullptr;
+    f.direct_vals = nullptr;
+    f.direct_cap = 0;
+    const bool stop = segment_flush(team, wb, ctl, f, writer);
+    wb.count = 0;
+    wb.thr = 0ull;
+    if (stop) return true;
+    if (cur_r < r_last) C = request_reference(a, team, ctl, cur_r + 1, ref_slot ^= 1);
+    ++cur_r;
+    return false;
+  };
+
+  bool stopped = false;
+  for (int i = 0; i < seq_count && !stopped; ++i) {
+    const int64_t row = seq_first + seq_stride * i;
+    const int r = static_cast<int>(row / a.B_in);
+    while (r > cur_r && !stopped) stopped = flush();
+    if (stopped) break;
+    if (!a.coop && a.layout) {
+      // A parent with very many children waits for the segment end, where all
+      // warps of the CTA walk it together (one warp alone would hold the CTA).
+      const int32_t pn = a.parent_nodes[row];
+      if (pn >= 0 && a.parent_scores[row] != __int_as_float(0xFF800000) &&
+          a.off[pn + 1] - a.off[pn] > kHeavyChildren) {
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(heavy_count, 1);
+        slot = __shfl_sync(kFull, slot, 0);
+        if (slot < kHeavyList) {
+          if (lane == 0) heavy[slot] = row;
+          continue;
+        }
+      }
+    }
+    do_row(row, r, part, nparts);
   }
   if (!stopped)
     while (cur_r <= r_last)
@@ -456,7 +488,7 @@ int launch_fused_lmhead(const sidbeam_trie* trie, int step, const void* hidden,
   while (npow2 < n_out) npow2 <<= 1;
   s.Cw = std::max((n_out + 31) / 32 * 32 + 32, (npow2 + kSelWarps - 1) / kSelWarps / 32 * 32 + 32);
   s.coop = part.rows_per_cta < kSelWarps ? 1 : 0;
-  const size_t smem = ((sizeof(SelCtl) + 127) / 128) * 128 + 1024 + 8192 +
+  const size_t smem = ((sizeof(SelCtl) + 127) / 128) * 128 + 1024 + 8192 + kHeavyList * 8 + 128 +
                       static_cast<size_t>(kSelWarps) * s.Cw * 12;
   if (smem > static_cast<size_t>(kSmemBudget))
     return set_error(SIDBEAM_ERR_INVALID_ARG, "fused_lmhead_step: n_out=%d too large", n_out);
