@@ -238,6 +238,49 @@ def test_quantised_logits_many_ties_bit_exact(tcb, layout):
     np.testing.assert_allclose(g["score"], ref["score"], atol=TOL)
 
 
+# ---------------------------------------------------------------- parents with many children
+def _wide_catalog(seed, V, heavy, light):
+    """Two levels: `heavy` first codes with 513 .. 3000 children each and
+    `light` first codes with a handful, interleaved."""
+    rng = np.random.default_rng(seed)
+    firsts = rng.permutation(V)[:heavy + light]
+    rows = []
+    for i, a in enumerate(firsts):
+        k = int(rng.integers(513, 3001)) if i % 2 == 0 and i // 2 < heavy else int(rng.integers(1, 9))
+        for c in rng.choice(V, size=k, replace=False):
+            rows.append((a, c))
+    return np.array(rows, dtype=np.int64)
+
+
+@pytest.mark.parametrize("R,B_in,n,layout,dtype", [
+    (2, 1200, 256, 1, "bf16"),    # one request over many CTAs, dense masks
+    (2, 1200, 256, 2, "bf16"),    # the same, CSR
+    (2, 1200, 256, 2, "f32"),     # 16 KB rows, walked in shared memory
+    (160, 40, 32, 2, "bf16"),     # several requests per CTA, CSR
+    (160, 40, 32, 1, "f32"),      # several requests per CTA, dense masks, 16 KB rows
+])
+def test_parents_with_many_children(tcb, R, B_in, n, layout, dtype):
+    """Parents with more than 512 children (past each warp's first rows they
+    are walked by a whole CTA at the end of their request's segment) mixed
+    with light ones, V = 4096; every request against the oracle."""
+    V = 4096
+    cat = _wide_catalog(R * 31 + layout, V, 24, 24)
+    otrie = oracle.OracleTrie(cat, [V, V])
+    gtrie = tcb.sid_trie_build(cat, [V, V], [layout, layout])
+    rng = np.random.default_rng(R + B_in + layout)
+    M = R * B_in
+    z = (3.0 * rng.standard_normal((M, V))).astype(np.float32)
+    if dtype == "bf16":
+        z = host.bf16_bits_to_f32(host.f32_to_bf16_bits(z))
+    ps = np.concatenate([np.sort(rng.uniform(-6, -1, size=B_in))[::-1] for _ in range(R)])
+    ps = ps.astype(np.float32)
+    ps[rng.random(M) < 0.03] = -np.inf
+    pn = rng.integers(0, otrie.n_nodes(1), size=M).astype(np.int32)
+    g, ws = _one_step(tcb, gtrie, 1, z, ps, pn, R, B_in, n, V, dtype=dtype)
+    assert tcb.sidbeam_get_device_status(ws) == 0
+    compare_step(g, otrie, 1, z, ps, pn, R, B_in, n, V)
+
+
 # ---------------------------------------------------------------- randomised sweep
 @pytest.mark.parametrize("seed", range(40))
 def test_random_sweep(tcb, seed):

@@ -570,23 +570,32 @@ __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRe
 }
 
 // Counts the hits in the CTA histogram and/or offers them to the warp buffer
-// (MODE); when offering, a hit that falls below a threshold raised meanwhile
+// (mode); when offering, a hit that falls below a threshold raised meanwhile
 // is dropped. The logits of the hits are read from the row's stage (held
-// until the walk is done): one compact loop instead of a copy of the walk per
-// register vector.
+// until the walk is done). One body out of line for the three modes: these
+// paths run for a minority of rows, so their code is shared (it stays warm in
+// the instruction cache) and the caller hands over no register copy of the
+// row (the hit bits are all it needs). The warp buffer goes in by value and
+// its new state comes back.
 enum TakeMode { kTakeBinOffer = 0, kTakeBin = 1, kTakeOffer = 2 };
 
-template <int BF16, int MODE>
-__device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* zrow,
-                                          const uint32_t (&hp)[kRegVecs / 4],
-                                          const uint32_t* wmask, uint32_t* wprefix,
-                                          const RowCtx& c, float& zthr, WarpBuf& wb, SelCtl* ctl,
-                                          const ThrSinks& sinks, int lane) {
+struct TakeOut {
+  uint64_t thr;
+  int count;
+  int binned;
+};
+
+template <int BF16>
+__device__ __noinline__ TakeOut take_hits(const StepArgs& a, const uint8_t* zrow, uint32_t h0,
+                                          uint32_t h1, uint32_t h2, uint32_t h3,
+                                          const uint32_t* wmask, uint32_t* wprefix, RowCtx c,
+                                          float zthr, WarpBuf wb, SelCtl* ctl, ThrSinks sinks,
+                                          int lane, int mode) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   constexpr int kBatch = 4;
   const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  if (dense && MODE != kTakeBin) dense_prefix(wmask, a.mask_words, wprefix, lane);
-  uint32_t hb[kRegVecs / 4] = {hp[0], hp[1], hp[2], hp[3]};
+  if (dense && mode != kTakeBin) dense_prefix(wmask, a.mask_words, wprefix, lane);
+  uint32_t hb[kRegVecs / 4] = {h0, h1, h2, h3};
   while (__any_sync(kFull, (hb[0] | hb[1] | hb[2] | hb[3]) != 0u)) {
     int code[kBatch];
     float z[kBatch];
@@ -603,17 +612,38 @@ __device__ __forceinline__ void take_hits(const StepArgs& a, const uint8_t* zrow
     for (int u = 0; u < kBatch; ++u) z[u] = code[u] >= 0 ? elem<BF16>(zrow, code[u]) : 0.f;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const bool has = code[u] >= 0 && (MODE == kTakeBin || z[u] >= zthr);
+      const bool has = code[u] >= 0 && (mode == kTakeBin || z[u] >= zthr);
       if (!__any_sync(kFull, has)) continue;
       const float score = c.s + (z[u] - c.lse);
-      if (MODE != kTakeOffer)
+      if (mode != kTakeOffer)
         warp_bin(ctl->hist, has, score_bin(score, c.C), wb.binned, &ctl->hist_total);
-      if (MODE != kTakeBin) {
+      if (mode != kTakeBin) {
         const int32_t node = (has && dense) ? dense_child(wmask, wprefix, c.o0, code[u]) : -1;
         warp_offer_nc(wb, has, make_key(score, c.idx0 + static_cast<uint32_t>(code[u])), node,
                       static_cast<uint32_t>(a.n), lane, sinks);
         zthr = zthreshold(wb.thr, c.s, c.lse);
       }
+    }
+  }
+  return TakeOut{wb.thr, wb.count, wb.binned};
+}
+
+// Drops the hits below zthr (hit logits read back from the stage).
+template <int BF16>
+__device__ __forceinline__ void hits_above(const uint8_t* zrow, uint32_t (&hp)[kRegVecs / 4],
+                                           float zthr, int lane) {
+  constexpr int kPerVec = BF16 ? 8 : 4;
+  const uint4* zq = reinterpret_cast<const uint4*>(zrow);
+#pragma unroll
+  for (int k = 0; k < kRegVecs; ++k) {
+    const uint32_t hb = (hp[k >> 2] >> ((k & 3) * 8)) & 0xFFu;
+    if (hb) {
+      const uint4 q = zq[lane + 32 * k];
+      uint32_t keep = 0u;
+#pragma unroll
+      for (int j = 0; j < kPerVec; ++j)
+        if (((hb >> j) & 1u) && vec_elem<BF16>(q, j) >= zthr) keep |= 1u << j;
+      hp[k >> 2] = (hp[k >> 2] & ~(0xFFu << ((k & 3) * 8))) | (keep << ((k & 3) * 8));
     }
   }
 }
@@ -1058,30 +1088,29 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         }
         const int nhits = static_cast<int>(
             __reduce_add_sync(kFull, __popc(hp[0]) + __popc(hp[1]) + __popc(hp[2]) + __popc(hp[3])));
+        auto take = [&](int mode) {
+          const TakeOut o = take_hits<BF16>(a, zrow, hp[0], hp[1], hp[2], hp[3], my_mask, my_prefix,
+                                            c, zthr, wb, ctl, sinks, lane, mode);
+          wb.thr = o.thr;
+          wb.count = o.count;
+          wb.binned = o.binned;
+        };
         if (nhits <= kOnePassHits) {
-          take_hits<BF16, kTakeBinOffer>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks,
-                                         lane);
+          take(kTakeBinOffer);
         } else {
           // Many hits: count them all, raise the threshold (this CTA's histogram,
           // then the request's), and offer only the hits that still reach it.
-          take_hits<BF16, kTakeBin>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks, lane);
+          take(kTakeBin);
           __syncwarp();
           refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
           if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
             push_histogram(a, ctl, r, C, wb, sinks, lane);
           const float zthr1 = zthreshold(wb.thr, c.s, c.lse);
-          if (zthr1 > zthr) {
-            // hits at the raised threshold: a subset of the ones counted
-#pragma unroll
-            for (int i = 0; i < kRegVecs / 4; ++i) hp[i] = 0u;
+          if (zthr1 > zthr) {  // hits at the raised threshold: a subset of the ones counted
             zthr = zthr1;
-            if (full && nparts == 1)
-              reg_hits<BF16, true>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
-            else
-              reg_hits<BF16, false>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
+            hits_above<BF16>(zrow, hp, zthr, lane);
           }
-          take_hits<BF16, kTakeOffer>(a, zrow, hp, my_mask, my_prefix, c, zthr, wb, ctl, sinks,
-                                      lane);
+          take(kTakeOffer);
         }
         release();
       }
