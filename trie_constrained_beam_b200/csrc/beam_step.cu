@@ -441,6 +441,36 @@ struct Ring {
 // stage's earlier contents were read by this warp's lanes: __syncwarp orders
 // those reads before lane 0, and the proxy fence before the async copy.
 // Returns false when the sequence has no live row left. Warp-collective.
+// Issues row `row` (sequence entry seq, parent data s, p, o0..o1) into the
+// stage just released: its logits and, behind them, its trie data.
+__device__ __forceinline__ void ring_issue(const StepArgs& a, Ring& g, int lane, uint64_t pol,
+                                           int seq, int64_t row, float s, int32_t p, uint32_t o0,
+                                           uint32_t o1) {
+  const int stage = g.issued % g.S;
+  if (lane == stage) {
+    g.st_seq = seq;
+    g.st_live = 1;
+    g.st_s = s;
+    g.st_p = p;
+    g.st_o0 = o0;
+    g.st_o1 = o1;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    uint8_t* dst = g.stages + static_cast<size_t>(stage) * a.cfg.stage_bytes;
+    const uint32_t ex = extra_bytes(a, o0, o1);
+    mbar_arrive_expect_tx(&g.full[stage], static_cast<uint32_t>(a.cfg.logits_copy_bytes) + ex);
+    bulk_copy_g2s(dst, a.logits + row * a.row_bytes,
+                  static_cast<uint32_t>(a.cfg.logits_copy_bytes), &g.full[stage], pol);
+    if (ex) copy_extra(a, dst, &g.full[stage], p, o0, ex, pol);
+  }
+  ++g.issued;
+}
+
+// Puts the next live row of the warp's own sequence into the stage just
+// released (parent data read 32 entries at a time). Returns false when the
+// sequence is exhausted.
 __device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, MetaBatch& mb,
                                            Ring& g, int lane, uint64_t pol) {
   while (g.ip < q.count) {
@@ -456,30 +486,31 @@ __device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, 
     const uint32_t o0 = __shfl_sync(kFull, mb.o0, j);
     const uint32_t o1 = __shfl_sync(kFull, mb.o1, j);
     const int seq = mb.base + j;
-    const int stage = g.issued % g.S;
-    if (lane == stage) {
-      g.st_seq = seq;
-      g.st_live = 1;
-      g.st_s = s;
-      g.st_p = p;
-      g.st_o0 = o0;
-      g.st_o1 = o1;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      uint8_t* dst = g.stages + static_cast<size_t>(stage) * a.cfg.stage_bytes;
-      const uint32_t ex = extra_bytes(a, o0, o1);
-      mbar_arrive_expect_tx(&g.full[stage], static_cast<uint32_t>(a.cfg.logits_copy_bytes) + ex);
-      bulk_copy_g2s(dst, a.logits + q.row(seq) * a.row_bytes,
-                    static_cast<uint32_t>(a.cfg.logits_copy_bytes), &g.full[stage], pol);
-      if (ex) copy_extra(a, dst, &g.full[stage], p, o0, ex, pol);
-    }
+    ring_issue(a, g, lane, pol, seq, q.row(seq), s, p, o0, o1);
     g.ip = seq + 1;
-    ++g.issued;
     return true;
   }
   return false;
+}
+
+// The same from the CTA's shared row table: the next entry of the CTA's
+// sequence goes to whichever warp asks first, so that a warp held up by a
+// heavy row takes fewer rows. Dead entries (score -inf in the table) are
+// skipped. cq: the CTA's whole sequence.
+__device__ __forceinline__ bool ring_refill_shared(const StepArgs& a, const RowSeq& cq,
+                                                  const uint4* meta, int* next, Ring& g, int lane,
+                                                  uint64_t pol) {
+  for (;;) {
+    int j = 0;
+    if (lane == 0) j = atomicAdd(next, 1);
+    j = __shfl_sync(kFull, j, 0);
+    if (j >= cq.count) return false;
+    const uint4 m = meta[j];
+    const float s = __uint_as_float(m.x);
+    if (s == __int_as_float(0xFF800000)) continue;
+    ring_issue(a, g, lane, pol, j, cq.row(j), s, static_cast<int32_t>(m.y), m.z, m.w);
+    return true;
+  }
 }
 
 // --------------------------------------------------------------- row walks
@@ -779,6 +810,10 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
   }
 }
 
+// Rows of a CTA whose parent data fits the shared table: up to this many, the
+// warps take rows from a shared counter instead of a fixed share each.
+constexpr int kMetaRows = 256;
+
 // Counts a CTA keeps before it moves them to the request's histogram.
 constexpr unsigned kPushAfter = 64;
 
@@ -817,20 +852,26 @@ __device__ void push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C, W
 // request (every child score is at most its parent's score), the same value
 // in every CTA. Two slots alternate so that one can be cleared while the
 // other is read. All team threads call it.
-__device__ __forceinline__ float segment_ref(const StepArgs& a, const Team& t, SelCtl* ctl, int r,
-                                             int slot) {
-  float m = __int_as_float(0xFF800000);
-  const float* ps = a.parent_scores + static_cast<int64_t>(r) * a.B_in;
-  for (int i = t.tid; i < a.B_in; i += t.T) {
-    const float x = ps[i];
-    if (x > __int_as_float(0xFF800000) && x < __int_as_float(0x7F800000)) m = fmaxf(m, x);
-  }
+__device__ __forceinline__ float finite_or_ninf(float x) {
+  return (x > __int_as_float(0xFF800000) && x < __int_as_float(0x7F800000))
+             ? x
+             : __int_as_float(0xFF800000);
+}
+// The reduction of the per-thread maxima m over the team.
+__device__ __forceinline__ float segment_ref_finish(const Team& t, SelCtl* ctl, int slot, float m) {
   m = warp_max(m);
   if (t.lane == 0 && m > __int_as_float(0xFF800000)) atomicMax(&ctl->ref_ord[slot], ord_f32(m));
   team_sync(t);
   const unsigned o = *reinterpret_cast<volatile unsigned*>(&ctl->ref_ord[slot]);
   if (t.tid == 0) ctl->ref_ord[slot ^ 1] = 0u;
   return o ? unord_f32(o) : 0.f;
+}
+__device__ __forceinline__ float segment_ref(const StepArgs& a, const Team& t, SelCtl* ctl, int r,
+                                             int slot) {
+  float m = __int_as_float(0xFF800000);
+  const float* ps = a.parent_scores + static_cast<int64_t>(r) * a.B_in;
+  for (int i = t.tid; i < a.B_in; i += t.T) m = fmaxf(m, finite_or_ninf(ps[i]));
+  return segment_ref_finish(t, ctl, slot, m);
 }
 
 // --------------------------------------------------------------- segment end
@@ -930,25 +971,14 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   }
   MetaBatch mb;
   load_meta(a, q, 0, lane, mb);
+  // Rows handed out from a shared table (the CTA's sequence; entries below
+  // W * S are the warps' first rows, issued above).
+  RowSeq cq;
+  a.part.rows(static_cast<int>(blockIdx.x), 0, 1, cq.first, cq.stride, cq.count);
+  const bool shared_rows = !a.coop && cq.count <= kMetaRows;
+  uint4* meta = reinterpret_cast<uint4*>(smem + cfg.off_meta);
 
-  // 2. CTA state, and the first segment's histogram reference.
-  if (threadIdx.x == 0) {
-    ctl->cta_thr = 0ull;
-    ctl->abort_flag = 0;
-    ctl->counter = 0;
-    ctl->ref_ord[0] = 0u;
-    ctl->ref_ord[1] = 0u;
-    ctl->hist_total = 0u;
-    ctl->push_lock = 0;
-  }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
-  __syncthreads();
-  const int r_first = static_cast<int>(lo / a.B_in);
-  const int r_last = static_cast<int>((hi - 1) / a.B_in);
-  int ref_slot = 0;
-  float C = segment_ref(a, team, ctl, r_first, ref_slot);
-
-  // 3. Trie data of the first rows, now that their parents are known.
+  // 2. Trie data of the first rows, now that their parents are known.
   for (int k = 0; k < spec; ++k) {
     const int live = (mb.live >> k) & 1u;
     const float s = __shfl_sync(kFull, mb.s, k);
@@ -956,7 +986,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     const uint32_t o0 = __shfl_sync(kFull, mb.o0, k);
     const uint32_t o1 = __shfl_sync(kFull, mb.o1, k);
     if (lane == k) {
-      g.st_seq = k;
+      g.st_seq = shared_rows ? warp + W * k : k;
       g.st_live = live;
       g.st_s = s;
       g.st_p = p;
@@ -973,11 +1003,69 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   g.issued = spec;
   g.ip = spec;
 
+  // 3. CTA state, the shared row table, and the first segment's histogram
+  //    reference.
+  if (threadIdx.x == 0) {
+    ctl->cta_thr = 0ull;
+    ctl->abort_flag = 0;
+    ctl->counter = 0;
+    ctl->ref_ord[0] = 0u;
+    ctl->ref_ord[1] = 0u;
+    ctl->hist_total = 0u;
+    ctl->push_lock = 0;
+    ctl->next_row = W * S;
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
+  __syncthreads();
+  const int r_first = static_cast<int>(lo / a.B_in);
+  const int r_last = static_cast<int>((hi - 1) / a.B_in);
+  int ref_slot = 0;
+  // The shared table (parent data of every row, as load_meta reads it; dead
+  // rows get score -inf) and the first segment's reference, their loads in
+  // flight together; the reference's barrier also publishes the table.
+  float mref = __int_as_float(0xFF800000);
+  {
+    const float* ps = a.parent_scores + static_cast<int64_t>(r_first) * a.B_in;
+    const int T = static_cast<int>(blockDim.x);
+    const int nt = shared_rows ? cq.count : 0;
+    for (int i0 = threadIdx.x; i0 < (nt > a.B_in ? nt : a.B_in); i0 += T) {
+      float sj = __int_as_float(0xFF800000);
+      int32_t pj = 0;
+      int64_t row = 0;
+      if (i0 < nt) {
+        row = cq.row(i0);
+        sj = a.parent_scores[row];
+        if (a.layout) pj = a.parent_nodes[row];
+      }
+      if (i0 < a.B_in) mref = fmaxf(mref, finite_or_ninf(ps[i0]));
+      if (i0 < nt) {
+        uint32_t o0 = 0u, o1 = 0u;
+        if (a.layout && (pj < 0 || static_cast<int64_t>(pj) >= a.n_parent)) {
+          if (pj >= 0 && sj != __int_as_float(0xFF800000)) atomicOr(a.status, kStatusBadNode);
+          sj = __int_as_float(0xFF800000);
+        } else if (a.layout && sj != __int_as_float(0xFF800000)) {
+          o0 = a.off[pj];
+          o1 = a.off[pj + 1];
+        }
+        meta[i0] = make_uint4(__float_as_uint(sj), static_cast<uint32_t>(pj), o0, o1);
+      }
+    }
+  }
+  float C = segment_ref_finish(team, ctl, ref_slot, mref);
+  if (shared_rows) q = cq;  // sequence entries are CTA entries from here on
+
   WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw,
              wvals + static_cast<size_t>(warp) * cfg.Cw, whist + warp * 256, cfg.Cw, 0, 0ull, 0};
   uint32_t* my_prefix = wprefix + warp * cfg.prefix_words;
   uint32_t* my_mask = wmask + warp * cfg.prefix_words;
   const int direct_cap = (W * S * cfg.stage_bytes / 12) & ~1;
+
+  auto refill = [&]() {
+    if (shared_rows)
+      ring_refill_shared(a, q, meta, &ctl->next_row, g, lane, pol);
+    else
+      ring_refill(a, q, mb, g, lane, pol);
+  };
 
   // End of the segment of request cur_r (all warps, in the same order).
   int cur_r = r_first;
@@ -1010,7 +1098,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     const uint8_t* zrow = g.stages + static_cast<size_t>(stage) * cfg.stage_bytes;
     if (!live) {
       ++g.consumed;
-      ring_refill(a, q, mb, g, lane, pol);
+      refill();
       continue;
     }
     const int64_t row = q.row(seq);
@@ -1051,7 +1139,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         held = false;
         __syncwarp();
         ++g.consumed;
-        ring_refill(a, q, mb, g, lane, pol);
+        refill();
         req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
         req_pref_r = r;
       };
@@ -1129,7 +1217,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
       if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
         push_histogram(a, ctl, r, C, wb, sinks, lane);
       ++g.consumed;
-      ring_refill(a, q, mb, g, lane, pol);
+      refill();
       req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
       req_pref_r = r;
     }
@@ -1190,6 +1278,8 @@ bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int
       o += ctl_bytes;
       c.off_bars = o;
       o += round_up(W * kMaxStages * 8, 128);
+      c.off_meta = o;
+      o += kMetaRows * 16;
       c.off_chist = o;
       o += 1024;
       c.off_whist = o;

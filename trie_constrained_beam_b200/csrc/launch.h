@@ -157,8 +157,8 @@ struct StepConfig {
   int extra_bytes;        // per stage after the row: dense mask row or staged CSR codes
   int prefix_words;       // dense levels: mask words per warp (prefix counts, mask copy)
   int reg;                // rows held in registers (<= 8 KB per row)
-  int off_ctl, off_bars, off_chist, off_whist, off_wprefix, off_wmask, off_stage, off_wkeys,
-      off_wvals;
+  int off_ctl, off_bars, off_meta, off_chist, off_whist, off_wprefix, off_wmask, off_stage,
+      off_wkeys, off_wvals;
   int smem_bytes;
 };
 

@@ -299,6 +299,7 @@ struct SelCtl {
   int rank_bad;                // rank merge: the entries did not match the histogram
   unsigned hist_total;         // candidates counted in `hist` and not yet pushed
   int push_lock;               // beam_step: one warp at a time moves `hist` to the request's
+  int next_row;                // beam_step: next entry of the CTA's row table to hand out
   unsigned ref_ord[2];         // beam_step: max parent score (ordered) of a segment, by parity
   int wcount[32];
   int segoff[kMaxSegCounts + 1];
