@@ -48,10 +48,10 @@ constexpr int kRegVecs = 16;  // 16-byte vectors per lane held in registers (8 K
 // A register row with more hits than this is walked in two passes (count,
 // raise the threshold, offer).
 constexpr int kOnePassHits = 64;
-// Dense rows with more children than this are walked in place in their stage
-// (counting there goes a vector at a time).
-constexpr uint32_t kHugeDense = 2048;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
+// Dense rows with more children than this, when every warp of the CTA takes
+// the row, are walked in place in their stage.
+constexpr uint32_t kHugeDense = 2048;
 
 // f(I) for I = 0 .. N-1 with I a compile-time constant (keeps register arrays
 // indexed statically).
@@ -576,34 +576,61 @@ __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRe
                                          float zthr, const uint32_t* wmask, int lane, int part,
                                          int nparts, uint32_t (&hp)[kRegVecs / 4]) {
   constexpr int kPerVec = BF16 ? 8 : 4;
-  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
+  const bool dense = wmask != nullptr;
 #pragma unroll
   for (int i = 0; i < kRegVecs / 4; ++i) hp[i] = 0u;
-  Unrolled<kRegVecs>::run([&](auto kc) {
-    constexpr int k = decltype(kc)::value;
-    const int v = lane + 32 * k;
-    const bool mine = FULL || (32 * k < nvec && (k % nparts) == part && v < nvec);
-    if (mine && vec_max<BF16>(x[k]) >= zthr) {
-      const int cb = v * kPerVec;
-      unsigned valid = (1u << kPerVec) - 1u;
-      if (dense)
-        valid = BF16 ? static_cast<unsigned>(reinterpret_cast<const uint8_t*>(wmask)[v])
-                     : (wmask[v >> 3] >> ((v & 7) * 4)) & 0xFu;
-      if (!FULL && a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
-      unsigned bits = 0u;
+  if (dense) {
+    // Masked rows: most vectors hold no valid child, so the mask decides
+    // first (one shared byte per vector), and only the valid codes of the
+    // remaining vectors are compared.
+    unsigned vm[kRegVecs];
 #pragma unroll
-      for (int j = 0; j < kPerVec; ++j)
-        if (((valid >> j) & 1u) && vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
-      hp[k >> 2] |= bits << ((k & 3) * 8);
+    for (int k = 0; k < kRegVecs; ++k) {
+      const int v = lane + 32 * k;
+      const bool mine = FULL || (32 * k < nvec && (k % nparts) == part && v < nvec);
+      vm[k] = !mine ? 0u
+                    : BF16 ? static_cast<unsigned>(reinterpret_cast<const uint8_t*>(wmask)[v])
+                           : (wmask[v >> 3] >> ((v & 7) * 4)) & 0xFu;
+      if (!FULL && a.V - v * kPerVec < kPerVec) vm[k] &= (1u << (a.V - v * kPerVec)) - 1u;
     }
-  });
+    Unrolled<kRegVecs>::run([&](auto kc) {
+      constexpr int k = decltype(kc)::value;
+      unsigned valid = vm[k];
+      if (valid && vec_max<BF16>(x[k]) >= zthr) {
+        unsigned bits = 0u;
+        while (valid) {
+          const int j = __ffs(valid) - 1;
+          valid &= valid - 1u;
+          if (vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
+        }
+        hp[k >> 2] |= bits << ((k & 3) * 8);
+      }
+    });
+  } else {
+    Unrolled<kRegVecs>::run([&](auto kc) {
+      constexpr int k = decltype(kc)::value;
+      const int v = lane + 32 * k;
+      const bool mine = FULL || (32 * k < nvec && (k % nparts) == part && v < nvec);
+      if (mine && vec_max<BF16>(x[k]) >= zthr) {
+        const int cb = v * kPerVec;
+        unsigned valid = (1u << kPerVec) - 1u;
+        if (!FULL && a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+        unsigned bits = 0u;
+#pragma unroll
+        for (int j = 0; j < kPerVec; ++j)
+          if (((valid >> j) & 1u) && vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
+        hp[k >> 2] |= bits << ((k & 3) * 8);
+      }
+    });
+  }
   return __any_sync(kFull, (hp[0] | hp[1] | hp[2] | hp[3]) != 0u);
 }
 
 // Counts the hits in the CTA histogram and/or offers them to the warp buffer
 // (mode); when offering, a hit that falls below a threshold raised meanwhile
-// is dropped. The logits of the hits are read from the row's stage (held
-// until the walk is done). One body out of line for the three modes: these
+// is dropped. The logits of the hits are read from zrow: the row in global
+// memory (or its stage, while that is held). One body out of line for the
+// three modes: these
 // paths run for a minority of rows, so their code is shared (it stays warm in
 // the instruction cache) and the caller hands over no register copy of the
 // row (the hit bits are all it needs). The warp buffer goes in by value and
@@ -624,8 +651,10 @@ __device__ __noinline__ TakeOut take_hits(const StepArgs& a, const uint8_t* zrow
                                           int lane, int mode) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   constexpr int kBatch = 4;
-  const bool dense = a.layout == SIDBEAM_LAYOUT_DENSE;
-  if (dense && mode != kTakeBin) dense_prefix(wmask, a.mask_words, wprefix, lane);
+  const bool dense = wmask != nullptr;  // node ids by rank in the child bitmap
+  if (dense && mode != kTakeBin)
+    dense_prefix(wmask, a.layout == SIDBEAM_LAYOUT_DENSE ? a.mask_words : (a.V + 31) / 32,
+                 wprefix, lane);
   uint32_t hb[kRegVecs / 4] = {h0, h1, h2, h3};
   while (__any_sync(kFull, (hb[0] | hb[1] | hb[2] | hb[3]) != 0u)) {
     int code[kBatch];
@@ -659,25 +688,6 @@ __device__ __noinline__ TakeOut take_hits(const StepArgs& a, const uint8_t* zrow
   return TakeOut{wb.thr, wb.count, wb.binned};
 }
 
-// Drops the hits below zthr (hit logits read back from the stage).
-template <int BF16>
-__device__ __forceinline__ void hits_above(const uint8_t* zrow, uint32_t (&hp)[kRegVecs / 4],
-                                           float zthr, int lane) {
-  constexpr int kPerVec = BF16 ? 8 : 4;
-  const uint4* zq = reinterpret_cast<const uint4*>(zrow);
-#pragma unroll
-  for (int k = 0; k < kRegVecs; ++k) {
-    const uint32_t hb = (hp[k >> 2] >> ((k & 3) * 8)) & 0xFFu;
-    if (hb) {
-      const uint4 q = zq[lane + 32 * k];
-      uint32_t keep = 0u;
-#pragma unroll
-      for (int j = 0; j < kPerVec; ++j)
-        if (((hb >> j) & 1u) && vec_elem<BF16>(q, j) >= zthr) keep |= 1u << j;
-      hp[k >> 2] = (hp[k >> 2] & ~(0xFFu << ((k & 3) * 8))) | (keep << ((k & 3) * 8));
-    }
-  }
-}
 
 // Child bitmap of a CSR node in the warp's mask copy: bit c set for every
 // child code c (child ids o0 .. o1-1, codes ascending, so the rank of a code
@@ -823,11 +833,11 @@ constexpr unsigned kPushAfter = 64;
 // skip). Counts move by atomic exchange, so each candidate stays counted
 // exactly once; the segment end pushes what is left. Only for requests split
 // over several CTAs (a CTA that holds a whole request keeps its histogram).
-__device__ void push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C, WarpBuf& wb,
-                               const ThrSinks& sinks, int lane) {
+__device__ __noinline__ uint64_t push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C,
+                                                uint64_t thr, ThrSinks sinks, int lane) {
   int got = 0;
   if (lane == 0) got = atomicCAS(&ctl->push_lock, 0, 1) == 0 ? 1 : 0;
-  if (!__shfl_sync(kFull, got, 0)) return;
+  if (!__shfl_sync(kFull, got, 0)) return thr;
   uint32_t* gh = a.ghist + static_cast<size_t>(r) * kHistBins;
   for (int b = lane; b < kHistBins; b += 32) {
     const uint32_t c = atomicExch(&ctl->hist[b], 0u);
@@ -840,12 +850,33 @@ __device__ void push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C, W
 #pragma unroll
   for (int j = 0; j < 8; ++j) h[j] = __ldcg(g4 + j);
   const uint64_t hb = hist_bound_regs(h, static_cast<uint32_t>(a.n), C, lane);
-  if (hb > wb.thr) {
-    wb.thr = hb;
+  if (hb > thr) {
+    thr = hb;
     publish_thr(hb, lane, sinks);
   }
   __syncwarp();
   if (lane == 0) atomicExch(&ctl->push_lock, 0);
+  return thr;
+}
+
+// refresh_thr with the histogram scan out of line (the scan runs for a
+// minority of rows; the cheap test stays inline).
+__device__ __noinline__ uint64_t refresh_scan(SelCtl* ctl, uint32_t n, float C, uint64_t thr,
+                                              ThrSinks sinks, int lane) {
+  WarpBuf wb{nullptr, nullptr, nullptr, 0, 0, thr, kRefreshAfter};
+  refresh_thr(wb, ctl, n, C, lane, sinks);
+  return wb.thr;
+}
+__device__ __forceinline__ void refresh_row(WarpBuf& wb, SelCtl* ctl, uint32_t n, float C,
+                                            int lane, const ThrSinks& sinks) {
+  if ((wb.binned < kRefreshAfter && wb.thr != 0ull) ||
+      *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) < n) {
+    const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+    if (c > wb.thr) wb.thr = c;
+    return;
+  }
+  wb.binned = 0;
+  wb.thr = refresh_scan(ctl, n, C, wb.thr, sinks, lane);
 }
 
 // Histogram reference of request r: the largest finite parent score of the
@@ -915,6 +946,46 @@ __device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf w
   const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
                           static_cast<uint32_t>(a.V)};
   return segment_flush(team, wb, ctl, f, writer);
+}
+
+// --------------------------------------------------------------- threshold seeding
+// The first row of every warp starts without a threshold, and together these
+// rows hold most of a step's candidates at levels where nodes have many
+// children. So before the per-row loop each warp counts every valid child of
+// its first row into a scratch histogram (exact scores, all lanes busy: no
+// per-candidate warp work); once all have counted, the n-th best of these
+// candidates bounds the request's n-th best from below and becomes the CTA's
+// and the request's first threshold. The scratch is not the segment
+// histogram, whose counts must match the candidates offered. Warp-collective;
+// zrow: the row's stage.
+template <int BF16>
+__device__ void seed_count(const StepArgs& a, const uint8_t* zrow, float s, float lse, uint32_t o0,
+                           uint32_t o1, float C, uint32_t* shist, int lane) {
+  constexpr int kPerVec = BF16 ? 8 : 4;
+  if (a.layout == SIDBEAM_LAYOUT_CSR) {
+    const uint32_t nst = csr_staged(a, o0, o1);
+    for (uint32_t k = o0 + lane; k < o1; k += 32u) {
+      const float z = elem<BF16>(zrow, csr_code(a, zrow, o0, nst, k));
+      atomicAdd(&shist[score_bin(s + (z - lse), C)], 1u);
+    }
+    return;
+  }
+  const uint32_t* mrow = a.layout == SIDBEAM_LAYOUT_DENSE
+                             ? reinterpret_cast<const uint32_t*>(zrow + a.cfg.logits_copy_bytes)
+                             : nullptr;
+  const uint4* q = reinterpret_cast<const uint4*>(zrow);
+  const int nvec = (a.V + kPerVec - 1) / kPerVec;
+  for (int v = lane; v < nvec; v += 32) {
+    const uint4 x = q[v];
+    const int cb = v * kPerVec;
+    unsigned valid = (1u << kPerVec) - 1u;
+    if (mrow) valid = (mrow[cb >> 5] >> (cb & 31)) & ((1u << kPerVec) - 1u);
+    if (a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
+#pragma unroll
+    for (int j = 0; j < kPerVec; ++j)
+      if ((valid >> j) & 1u)
+        atomicAdd(&shist[score_bin(s + (vec_elem<BF16>(x, j) - lse), C)], 1u);
+  }
 }
 
 // --------------------------------------------------------------- kernel
@@ -1015,7 +1086,10 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     ctl->push_lock = 0;
     ctl->next_row = W * S;
   }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) ctl->hist[i] = 0u;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+    ctl->hist[i] = 0u;
+    whist[i] = 0u;  // seeding scratch (the warps' select scratch later)
+  }
   __syncthreads();
   const int r_first = static_cast<int>(lo / a.B_in);
   const int r_last = static_cast<int>((hi - 1) / a.B_in);
@@ -1053,6 +1127,38 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   }
   float C = segment_ref_finish(team, ctl, ref_slot, mref);
   if (shared_rows) q = cq;  // sequence entries are CTA entries from here on
+
+  // 3b. Threshold seeding from the first row of every warp that belongs to
+  //     the first request, when those rows have more than n children in all
+  //     (read from the shared table).
+  if (shared_rows) {
+    const int64_t end_first = static_cast<int64_t>(r_first + 1) * a.B_in;  // rows of r_first
+    const int nfirst = cq.count < W ? cq.count : W;
+    uint32_t nch = 0u;
+    for (int j = lane; j < nfirst; j += 32) {
+      const uint4 m = meta[j];
+      if (m.x != 0xFF800000u && cq.row(j) < end_first)
+        nch += a.layout ? m.w - m.z : static_cast<uint32_t>(a.V);
+    }
+    if (warp_sum_u(nch) > static_cast<uint32_t>(a.n)) {  // the same in every warp
+      if (warp < cq.count && meta[warp].x != 0xFF800000u && cq.row(warp) < end_first &&
+          bounded_wait(&g.full[0], 0u, &ctl->abort_flag, a.status, kStatusTimeout)) {
+        const uint4 m = meta[warp];  // the warp's first row: CTA entry `warp`, stage 0
+        float rmax0, lse0;
+        row_stats<BF16>(g.stages, a.V, lane, rmax0, lse0);
+        seed_count<BF16>(a, g.stages, __uint_as_float(m.x), lse0, m.z, m.w, C, whist, lane);
+      }
+      team_sync(team);
+      if (warp == 0) {
+        const uint64_t hb = hist_bound(whist, static_cast<uint32_t>(a.n), C, lane);
+        if (lane == 0 && hb) {
+          atomicMax(&ctl->cta_thr, static_cast<unsigned long long>(hb));
+          atomicMax(a.request_thr + r_first, static_cast<unsigned long long>(hb));
+        }
+      }
+      team_sync(team);  // the scratch goes back to the warps
+    }
+  }
 
   WarpBuf wb{wkeys + static_cast<size_t>(warp) * cfg.Cw,
              wvals + static_cast<size_t>(warp) * cfg.Cw, whist + warp * 256, cfg.Cw, 0, 0ull, 0};
@@ -1113,8 +1219,13 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
     const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
     const uint32_t nchild = o1 - o0;
-    const bool reg_row = REG && (csr ? nchild <= static_cast<uint32_t>(32 * nparts)
-                                     : (a.layout != SIDBEAM_LAYOUT_DENSE || nchild <= kHugeDense));
+    // Register rows: all but CSR nodes with more children than one 32-lane
+    // batch per warp, and, when every warp takes every row (a CTA with fewer
+    // rows than warps), dense nodes with very many children; those are walked
+    // in place in their stage.
+    const bool reg_row =
+        REG && (csr ? nchild <= static_cast<uint32_t>(32 * nparts)
+                    : (a.layout != SIDBEAM_LAYOUT_DENSE || nparts == 1 || nchild <= kHugeDense));
     if (reg_row) {
       uint4 x[kRegVecs];
       copy_row_regs<BF16>(zrow, a.V, lane, x);
@@ -1131,19 +1242,15 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         ccode = csr_code(a, zrow, o0, csr_staged(a, o0, o1), ck);
         cz = elem<BF16>(zrow, ccode);
       }
-      // The stage goes back now at CSR levels (the walk needs nothing more from
-      // it); dense and unconstrained rows keep it until their walk is done.
-      bool held = true;
-      auto release = [&]() {
-        if (!held) return;
-        held = false;
-        __syncwarp();
-        ++g.consumed;
-        refill();
-        req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
-        req_pref_r = r;
-      };
-      if (csr) release();
+      // Everything the row needs from its stage is now in registers or in the
+      // warp's mask copy: the stage goes back at once, so that the next row's
+      // copy overlaps this row's arithmetic (the few hit logits a walk needs
+      // are read back from the row in global memory, still in L2).
+      __syncwarp();
+      ++g.consumed;
+      refill();
+      req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
+      req_pref_r = r;
 
       const int nvec = (a.V + kPerVec - 1) / kPerVec;
       const bool full = nvec == 32 * kRegVecs && a.V % kPerVec == 0;
@@ -1154,10 +1261,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
       float zthr = zthreshold(wb.thr, c.s, c.lse);
-      if (rmax < zthr) {
-        release();
-        continue;
-      }
+      if (rmax < zthr) continue;
       if (csr) {
         const bool ok = cin && cz >= zthr;
         if (!__any_sync(kFull, ok)) continue;
@@ -1166,19 +1270,19 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         warp_offer_nc(wb, ok, make_key(score, c.idx0 + static_cast<uint32_t>(ccode)),
                       static_cast<int32_t>(ck), static_cast<uint32_t>(a.n), lane, sinks);
       } else {
+        const uint32_t* hmask = a.layout == SIDBEAM_LAYOUT_DENSE ? my_mask : nullptr;
         uint32_t hp[kRegVecs / 4];
-        const bool any = (full && nparts == 1)
-                             ? reg_hits<BF16, true>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp)
-                             : reg_hits<BF16, false>(a, x, nvec, zthr, my_mask, lane, part, nparts, hp);
-        if (!any) {
-          release();
-          continue;
-        }
+        const bool any =
+            (full && nparts == 1)
+                ? reg_hits<BF16, true>(a, x, nvec, zthr, hmask, lane, part, nparts, hp)
+                : reg_hits<BF16, false>(a, x, nvec, zthr, hmask, lane, part, nparts, hp);
+        if (!any) continue;
         const int nhits = static_cast<int>(
             __reduce_add_sync(kFull, __popc(hp[0]) + __popc(hp[1]) + __popc(hp[2]) + __popc(hp[3])));
+        const uint8_t* zg = a.logits + row * a.row_bytes;
         auto take = [&](int mode) {
-          const TakeOut o = take_hits<BF16>(a, zrow, hp[0], hp[1], hp[2], hp[3], my_mask, my_prefix,
-                                            c, zthr, wb, ctl, sinks, lane, mode);
+          const TakeOut o = take_hits<BF16>(a, zg, hp[0], hp[1], hp[2], hp[3], hmask, my_prefix, c,
+                                            zthr, wb, ctl, sinks, lane, mode);
           wb.thr = o.thr;
           wb.count = o.count;
           wb.binned = o.binned;
@@ -1190,22 +1294,18 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
           // then the request's), and offer only the hits that still reach it.
           take(kTakeBin);
           __syncwarp();
-          refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+          refresh_row(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
           if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
-            push_histogram(a, ctl, r, C, wb, sinks, lane);
+            wb.thr = push_histogram(a, ctl, r, C, wb.thr, sinks, lane);
           const float zthr1 = zthreshold(wb.thr, c.s, c.lse);
-          if (zthr1 > zthr) {  // hits at the raised threshold: a subset of the ones counted
-            zthr = zthr1;
-            hits_above<BF16>(zrow, hp, zthr, lane);
-          }
+          if (zthr1 > zthr) zthr = zthr1;
           take(kTakeOffer);
         }
-        release();
       }
       __syncwarp();
-      refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+      refresh_row(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
       if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
-        push_histogram(a, ctl, r, C, wb, sinks, lane);
+        wb.thr = push_histogram(a, ctl, r, C, wb.thr, sinks, lane);
     } else {
       float rmax;
       row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
@@ -1213,9 +1313,9 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
       smem_walk<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
                       my_mask, sinks, lane, part, nparts);
       __syncwarp();
-      refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
+      refresh_row(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
       if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
-        push_histogram(a, ctl, r, C, wb, sinks, lane);
+        wb.thr = push_histogram(a, ctl, r, C, wb.thr, sinks, lane);
       ++g.consumed;
       refill();
       req_pref = *reinterpret_cast<volatile unsigned long long*>(a.request_thr + r);
