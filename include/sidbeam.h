@@ -163,6 +163,31 @@ int beam_step(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dt
               int32_t* out_code, int32_t* out_node, void* workspace, size_t workspace_bytes,
               void* stream);
 
+/* beam_step_ex -- beam_step with options (flags: OR of SIDBEAM_STEP_*).
+ *  SIDBEAM_STEP_SKIP_ROWS: row skipping (the first of the "next" items, not a
+ *  step the pages describe; it leaves every result unchanged). Every child's
+ *  score s + (z - lse) is at most its parent's score s (z <= lse), so a row
+ *  whose parent score cannot reach a valid lower bound on the request's n-th
+ *  best key that the step already holds can contribute nothing: its logits
+ *  are not read. Applies when the request's rows are spread over CTAs that
+ *  each hold only that request (R no larger than the GPU's SM count); the
+ *  first rows of each CTA are always read. The number of rows passed over
+ *  accumulates in the workspace (beam_step_skipped_rows).
+ *  Other arguments, results and errors: those of beam_step; unknown flag bits
+ *  give INVALID_ARG. beam_step(...) is beam_step_ex(..., 0). */
+#define SIDBEAM_STEP_SKIP_ROWS 1u
+int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dtype dtype,
+                 int64_t ld, const float* parent_scores, const int32_t* parent_nodes, int R,
+                 int B_in, int n_out, int V, float* out_scores, int32_t* out_parent,
+                 int32_t* out_code, int32_t* out_node, void* workspace, size_t workspace_bytes,
+                 void* stream, unsigned flags);
+
+/* beam_step_skipped_rows -- rows not read by row skipping since the last call
+ * on this workspace (host *count); the counter is reset to zero. `stream`
+ * orders the read after the steps that used the workspace (the call
+ * synchronises it). Errors: INVALID_ARG, CUDA. */
+int beam_step_skipped_rows(void* workspace, uint32_t* count, void* stream);
+
 /* beam_step_noalloc -- the same step as beam_step, for callers that cannot
  * allocate device memory when they run it (a plugin whose host application owns
  * every device allocation or enforces a fixed budget, a serving loop that plans

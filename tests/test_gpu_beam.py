@@ -281,6 +281,84 @@ def test_parents_with_many_children(tcb, R, B_in, n, layout, dtype):
     compare_step(g, otrie, 1, z, ps, pn, R, B_in, n, V)
 
 
+# ---------------------------------------------------------------- row skipping
+def _search_outputs(tcb, w, gtrie, skip_rows):
+    """The whole wide-beam search on the device generator's logits; every
+    step's outputs, plus the rows row skipping left unread."""
+    import torch
+    from sidgen import device as gdev
+    search = tcb.BeamSearch(gtrie, w.R, w.n, w.V, depth=w.depth, skip_rows=skip_rows)
+    hashes = torch.from_numpy(host.request_roots(w.R).view(np.int64)).to("cuda")
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    outs, skipped = [], []
+    for t in range(w.depth):
+        logits = torch.empty((search.rows(t), w.V), dtype=tdt, device="cuda")
+        gdev.row_logits(w.logits_seed, hashes, w.V, w.sigma, logits)
+        search.step(t, logits)
+        assert tcb.sidbeam_get_device_status(search.workspace) == 0
+        skipped.append(search.skipped_rows())
+        ps, pn, B_in = search.parents(t)
+        outs.append([x.cpu().numpy().copy() for x in (search.scores[t], search.bp_parent[t],
+                                                      search.bp_code[t], search.nodes[t])])
+        child = torch.empty((w.R * w.n,), dtype=torch.int64, device="cuda")
+        gdev.child_hash(hashes, w.R, B_in, search.bp_parent[t], search.bp_code[t], w.n, t + 1,
+                        child)
+        hashes = child
+    return outs, skipped
+
+
+def test_row_skipping_changes_no_result_wide_beam(tcb):
+    """The wide-beam search with row skipping on gives every step's outputs bit
+    for bit as with it off (both are checked against the oracle elsewhere). At
+    this workload the request's n-th best child stays below every parent's
+    score, so no row qualifies; the low-parents test below exercises skipping."""
+    w = WORKLOADS[4]
+    cat, _ = _catalog(4)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    ref, none = _search_outputs(tcb, w, gtrie, False)
+    got, skipped = _search_outputs(tcb, w, gtrie, True)
+    assert sum(none) == 0
+    for t in range(w.depth):
+        for a, b in zip(ref[t], got[t]):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), f"step {t}"
+    assert all(k >= 0 for k in skipped)
+
+
+def test_row_skipping_low_parents_oracle(tcb):
+    """Two requests of 2,000 parents (V = 4,096, bf16, 200 children each), the
+    first 100 of each with scores near 0 and the rest at -1000: once the first
+    rows have set a bound, the low rows are skipped; the result equals the
+    oracle's."""
+    import torch
+    V = 4096
+    rng = np.random.default_rng(3)
+    cat = np.array([(a, c) for a in range(100) for c in rng.choice(V, size=200, replace=False)])
+    otrie = oracle.OracleTrie(cat, [V, V])
+    gtrie = tcb.sid_trie_build(cat, [V, V], [2, 2])
+    R, B_in, n = 2, 2000, 64
+    M = R * B_in
+    z = host.bf16_bits_to_f32(host.f32_to_bf16_bits(
+        (2.0 * rng.standard_normal((M, V))).astype(np.float32)))
+    ps = np.full(M, -1000.0, np.float32)
+    for r in range(R):
+        ps[r * B_in:r * B_in + 100] = np.sort(rng.uniform(-1, 0, 100))[::-1]
+    pn = rng.integers(0, otrie.n_nodes(1), size=M).astype(np.int32)
+    out = dict(score=torch.empty(R * n, device="cuda"),
+               parent=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               code=torch.empty(R * n, dtype=torch.int32, device="cuda"),
+               node=torch.empty(R * n, dtype=torch.int32, device="cuda"))
+    ws = torch.zeros(tcb.beam_step_workspace_size(R, B_in, n, V), dtype=torch.uint8, device="cuda")
+    tcb.beam_step(gtrie, 1, torch.from_numpy(z).cuda().to(torch.bfloat16), torch.from_numpy(ps).cuda(),
+                  torch.from_numpy(pn).cuda(), R, B_in, n, V, out["score"], out["parent"],
+                  out["code"], out["node"], ws, skip_rows=True)
+    assert tcb.sidbeam_get_device_status(ws) == 0
+    skipped = tcb.beam_step_skipped_rows(ws)
+    assert skipped > 0
+    assert tcb.beam_step_skipped_rows(ws) == 0  # read and reset
+    g = {k: v.cpu().numpy().reshape(R, n) for k, v in out.items()}
+    compare_step(g, otrie, 1, z, ps, pn, R, B_in, n, V)
+
+
 # ---------------------------------------------------------------- randomised sweep
 @pytest.mark.parametrize("seed", range(40))
 def test_random_sweep(tcb, seed):

@@ -39,7 +39,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      const float* parent_scores, const int32_t* parent_nodes, int R, int B_in,
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream);
+                     cudaStream_t stream, unsigned flags);
 
 namespace {
 
@@ -95,6 +95,19 @@ extern "C" int beam_step(const sidbeam_trie* trie, int step, const void* logits,
                          float* out_scores, int32_t* out_parent, int32_t* out_code,
                          int32_t* out_node, void* workspace, size_t workspace_bytes,
                          void* stream) {
+  return beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in, n_out,
+                      V, out_scores, out_parent, out_code, out_node, workspace, workspace_bytes,
+                      stream, 0u);
+}
+
+extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
+                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                            float* out_scores, int32_t* out_parent, int32_t* out_code,
+                            int32_t* out_node, void* workspace, size_t workspace_bytes,
+                            void* stream, unsigned flags) {
+  if (flags & ~static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS))
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
   if (!logits || !parent_scores || !out_scores || !out_parent || !out_code || !out_node)
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: NULL pointer argument");
   if (trie && !parent_nodes)
@@ -131,7 +144,7 @@ extern "C" int beam_step(const sidbeam_trie* trie, int step, const void* logits,
     return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step: workspace must be 256-byte aligned");
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
-                          workspace_bytes, static_cast<cudaStream_t>(stream));
+                          workspace_bytes, static_cast<cudaStream_t>(stream), flags);
 }
 
 extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,
@@ -149,6 +162,24 @@ extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,
       depth, R, n, bp_parent, bp_code, last_node, out_sids, out_leaf);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SIDBEAM_OK : cuda_error(e, "beam_finalize: launch");
+}
+
+extern "C" int beam_step_skipped_rows(void* workspace, uint32_t* count, void* stream) {
+  if (!workspace || !count)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step_skipped_rows: NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace) + kSkippedRowsOffset;
+  uint32_t c = 0;
+  cudaError_t e = cudaMemcpyAsync(&c, w, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && c) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyAsync(w, &zero, 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return cuda_error(e, "beam_step_skipped_rows");
+  *count = c;
+  return SIDBEAM_OK;
 }
 
 extern "C" int sidbeam_get_device_status(void* workspace, void* stream) {

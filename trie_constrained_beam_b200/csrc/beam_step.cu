@@ -98,6 +98,8 @@ struct StepArgs {
   Partition part;
   StepConfig cfg;
   int coop;  // 1: every warp takes every row of the CTA (fewer rows than warps)
+  int skip_rows;     // 1: rows whose parent score is below the request's bound are not read
+  uint32_t* skipped; // counter of rows not read for that reason
 };
 
 struct StepWriter {
@@ -441,6 +443,16 @@ struct Ring {
 // stage's earlier contents were read by this warp's lanes: __syncwarp orders
 // those reads before lane 0, and the proxy fence before the async copy.
 // Returns false when the sequence has no live row left. Warp-collective.
+// Row skipping (optional). Every child score s + (z - lse) is at most the
+// parent score s in fp32 (z <= lse, so z - lse <= 0 after rounding, and
+// adding a non-positive number does not raise s), so the largest key a child
+// of the row can have is key(s, lowest index). When that is below a valid
+// lower bound on the request's n-th best key, no child of the row can be
+// selected and its logits need not be read: the result is the same.
+__device__ __forceinline__ bool row_skippable(float s, uint64_t bound) {
+  return bound != 0ull && make_key(s, 0u) < bound;
+}
+
 // Issues row `row` (sequence entry seq, parent data s, p, o0..o1) into the
 // stage just released: its logits and, behind them, its trie data.
 __device__ __forceinline__ void ring_issue(const StepArgs& a, Ring& g, int lane, uint64_t pol,
@@ -470,9 +482,10 @@ __device__ __forceinline__ void ring_issue(const StepArgs& a, Ring& g, int lane,
 
 // Puts the next live row of the warp's own sequence into the stage just
 // released (parent data read 32 entries at a time). Returns false when the
-// sequence is exhausted.
+// sequence is exhausted. Rows that row_skippable rules out against `bound`
+// (0: none) are passed over and counted.
 __device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, MetaBatch& mb,
-                                           Ring& g, int lane, uint64_t pol) {
+                                           Ring& g, int lane, uint64_t pol, uint64_t bound) {
   while (g.ip < q.count) {
     if (g.ip >= mb.base + 32) load_meta(a, q, g.ip & ~31, lane, mb);
     const unsigned m = mb.live & (~0u << (g.ip - mb.base));
@@ -486,8 +499,12 @@ __device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, 
     const uint32_t o0 = __shfl_sync(kFull, mb.o0, j);
     const uint32_t o1 = __shfl_sync(kFull, mb.o1, j);
     const int seq = mb.base + j;
-    ring_issue(a, g, lane, pol, seq, q.row(seq), s, p, o0, o1);
     g.ip = seq + 1;
+    if (row_skippable(s, bound)) {
+      if (lane == 0) atomicAdd(a.skipped, 1u);
+      continue;
+    }
+    ring_issue(a, g, lane, pol, seq, q.row(seq), s, p, o0, o1);
     return true;
   }
   return false;
@@ -499,7 +516,7 @@ __device__ __forceinline__ bool ring_refill(const StepArgs& a, const RowSeq& q, 
 // skipped. cq: the CTA's whole sequence.
 __device__ __forceinline__ bool ring_refill_shared(const StepArgs& a, const RowSeq& cq,
                                                   const uint4* meta, int* next, Ring& g, int lane,
-                                                  uint64_t pol) {
+                                                  uint64_t pol, uint64_t bound) {
   for (;;) {
     int j = 0;
     if (lane == 0) j = atomicAdd(next, 1);
@@ -508,6 +525,10 @@ __device__ __forceinline__ bool ring_refill_shared(const StepArgs& a, const RowS
     const uint4 m = meta[j];
     const float s = __uint_as_float(m.x);
     if (s == __int_as_float(0xFF800000)) continue;
+    if (row_skippable(s, bound)) {
+      if (lane == 0) atomicAdd(a.skipped, 1u);
+      continue;
+    }
     ring_issue(a, g, lane, pol, j, cq.row(j), s, static_cast<int32_t>(m.y), m.z, m.w);
     return true;
   }
@@ -729,11 +750,17 @@ __device__ __forceinline__ void csr_bitmap(const StepArgs& a, uint32_t o0, uint3
 // more children than one 32-lane batch per warp, dense rows with very many
 // children). wmask: the warp's mask copy (room for a V-bit row).
 constexpr uint32_t kCsrBitmapMin = 192;  // CSR rows with more children use a bitmap
+// Counts a CTA keeps before it moves them to the request's histogram.
+constexpr unsigned kPushAfter = 64;
+__device__ __noinline__ uint64_t push_histogram(const StepArgs& a, SelCtl* ctl, int r, float C,
+                                                uint64_t thr, ThrSinks sinks, int lane);
+// r: the row's request; multi: the request is split over several CTAs (the
+// count pass then also pushes, so that the offer pass sees their counts).
 template <int BF16>
 __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
                           float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
                           uint32_t* wmask, const ThrSinks& sinks, int lane, int part,
-                          int nparts) {
+                          int nparts, int r, bool multi) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   if (rmax < zthr) return;  // even the row's largest logit cannot reach the threshold
   const uint32_t* mrow = nullptr;  // valid-child bitmap (null: every code is valid)
@@ -815,6 +842,8 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
     if (pass == 0) {
       __syncwarp();
       refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), c.C, lane, sinks);
+      if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
+        wb.thr = push_histogram(a, ctl, r, c.C, wb.thr, sinks, lane);
       zthr = zthreshold(wb.thr, c.s, c.lse);
     }
   }
@@ -823,9 +852,6 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
 // Rows of a CTA whose parent data fits the shared table: up to this many, the
 // warps take rows from a shared counter instead of a fixed share each.
 constexpr int kMetaRows = 256;
-
-// Counts a CTA keeps before it moves them to the request's histogram.
-constexpr unsigned kPushAfter = 64;
 
 // Moves this CTA's histogram counts into request r's global histogram and
 // raises the shared bounds from the global one, which holds every CTA's
@@ -1166,11 +1192,22 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   uint32_t* my_mask = wmask + warp * cfg.prefix_words;
   const int direct_cap = (W * S * cfg.stage_bytes / 12) & ~1;
 
+  // The request's shared bound as last read (after each row is issued).
+  unsigned long long req_pref = 0ull;
+  int req_pref_r = -1;
+  // Row skipping needs a bound of the rows' own request: CTAs that hold rows
+  // of one request only.
+  const bool skipping = a.skip_rows && a.part.grouped;
   auto refill = [&]() {
+    uint64_t bound = 0ull;
+    if (skipping) {
+      bound = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+      if (req_pref_r >= 0 && req_pref > bound) bound = req_pref;
+    }
     if (shared_rows)
-      ring_refill_shared(a, q, meta, &ctl->next_row, g, lane, pol);
+      ring_refill_shared(a, q, meta, &ctl->next_row, g, lane, pol, bound);
     else
-      ring_refill(a, q, mb, g, lane, pol);
+      ring_refill(a, q, mb, g, lane, pol, bound);
   };
 
   // End of the segment of request cur_r (all warps, in the same order).
@@ -1187,8 +1224,6 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   };
 
   bool wait_failed = false, stopped = false;
-  unsigned long long req_pref = 0ull;
-  int req_pref_r = -1;
   while (g.consumed < g.issued) {
     const int stage = g.consumed % S;
     if (!bounded_wait(&g.full[stage], (g.consumed / S) & 1u, &ctl->abort_flag, a.status,
@@ -1311,7 +1346,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
       row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
       row_thresholds(wb, ctl, req_now);
       smem_walk<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
-                      my_mask, sinks, lane, part, nparts);
+                      my_mask, sinks, lane, part, nparts, r, multi);
       __syncwarp();
       refresh_row(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
       if (multi && *reinterpret_cast<volatile unsigned*>(&ctl->hist_total) >= kPushAfter)
@@ -1433,7 +1468,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      const float* parent_scores, const int32_t* parent_nodes, int R, int B_in,
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, unsigned flags) {
   StepArgs a{};
   a.logits = static_cast<const uint8_t*>(logits);
   a.bf16 = dtype == SIDBEAM_BF16;
@@ -1467,6 +1502,8 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      workspace_bytes, ws.total);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<uint32_t*>(w + ws.status);
+  a.skipped = reinterpret_cast<uint32_t*>(w + ws.status + kSkippedRowsOffset);
+  a.skip_rows = (flags & SIDBEAM_STEP_SKIP_ROWS) ? 1 : 0;
   a.tickets = reinterpret_cast<uint32_t*>(w + ws.tickets);
   a.request_thr = reinterpret_cast<unsigned long long*>(w + ws.request_thr);
   a.part_count = reinterpret_cast<uint32_t*>(w + ws.part_count);

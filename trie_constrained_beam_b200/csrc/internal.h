@@ -49,5 +49,8 @@ int device_sm_count();
 // Device status word bits (first 4 bytes of a workspace).
 constexpr uint32_t kStatusBadNode = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
+// Byte offset, inside the workspace's first 256-byte block (after the status
+// word), of the counter of rows beam_step did not read (row skipping).
+constexpr size_t kSkippedRowsOffset = 8;
 
 }  // namespace sidbeam

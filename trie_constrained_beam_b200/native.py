@@ -42,8 +42,11 @@ EXPORTED = (
     "sid_trie_free", "beam_step_workspace_size", "beam_step", "beam_finalize",
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
     "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc", "lmhead_logits",
-    "fused_lmhead_workspace_size", "sidbeam_fused_lmhead_step",
+    "fused_lmhead_workspace_size", "sidbeam_fused_lmhead_step", "beam_step_ex",
+    "beam_step_skipped_rows",
 )
+
+STEP_SKIP_ROWS = 1  # SIDBEAM_STEP_SKIP_ROWS
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -77,6 +80,9 @@ def load():
     L.beam_step_workspace_size.restype = SZ
     L.beam_step.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
     L.beam_step_noalloc.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P]
+    L.beam_step_ex.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P,
+                               ctypes.c_uint]
+    L.beam_step_skipped_rows.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
     L.beam_finalize.argtypes = [I32, I32, I32, P, P, P, P, P, P]
     L.catalog_score_workspace_size.argtypes = [P, I32, I32]
     L.catalog_score_workspace_size.restype = SZ
@@ -93,7 +99,8 @@ def load():
     L.sidbeam_version.restype = ctypes.c_char_p
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
                  "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
-                 "sidbeam_get_device_status", "lmhead_logits", "sidbeam_fused_lmhead_step"):
+                 "sidbeam_get_device_status", "lmhead_logits", "sidbeam_fused_lmhead_step",
+                 "beam_step_ex", "beam_step_skipped_rows"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -197,17 +204,30 @@ def beam_step_workspace_size(R: int, B_in: int, n_out: int, V: int) -> int:
 
 
 def beam_step(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V,
-              out_scores, out_parent, out_code, out_node, workspace, stream=None, ld=None):
-    """logits: torch [R*B_in, ld] float32/bfloat16 on the device (row stride = ld)."""
+              out_scores, out_parent, out_code, out_node, workspace, stream=None, ld=None,
+              skip_rows=False):
+    """logits: torch [R*B_in, ld] float32/bfloat16 on the device (row stride = ld).
+    skip_rows: do not read rows that cannot contribute (beam_step_ex with
+    SIDBEAM_STEP_SKIP_ROWS); the results are the same."""
     if ld is None:
         ld = logits.stride(0)
-    rc = load().beam_step(None if trie is None else trie.handle, step, _ptr(logits),
-                          _dtype_code(logits), ld, _ptr(parent_scores), _ptr(parent_nodes), R,
-                          B_in, n_out, V, _ptr(out_scores), _ptr(out_parent), _ptr(out_code),
-                          _ptr(out_node), _ptr(workspace),
-                          0 if workspace is None else workspace.numel() * workspace.element_size(),
-                          _stream(stream))
+    args = (None if trie is None else trie.handle, step, _ptr(logits), _dtype_code(logits), ld,
+            _ptr(parent_scores), _ptr(parent_nodes), R, B_in, n_out, V, _ptr(out_scores),
+            _ptr(out_parent), _ptr(out_code), _ptr(out_node), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _stream(stream))
+    if skip_rows:
+        rc = load().beam_step_ex(*args, STEP_SKIP_ROWS)
+    else:
+        rc = load().beam_step(*args)
     _check(rc)
+
+
+def beam_step_skipped_rows(workspace, stream=None) -> int:
+    """Rows row skipping left unread since the last call (the counter resets)."""
+    c = ctypes.c_uint32(0)
+    _check(load().beam_step_skipped_rows(_ptr(workspace), ctypes.byref(c), _stream(stream)))
+    return int(c.value)
 
 
 def beam_step_noalloc(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V,

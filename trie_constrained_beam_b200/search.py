@@ -13,8 +13,10 @@ from . import native
 
 
 class BeamSearch:
-    def __init__(self, trie, R: int, n: int, V, depth: int = None, device="cuda"):
+    def __init__(self, trie, R: int, n: int, V, depth: int = None, device="cuda",
+                 skip_rows: bool = False):
         self.trie = trie
+        self.skip_rows = skip_rows  # beam_step_ex row skipping (same results)
         self.depth = depth if depth is not None else trie.depth
         self.V = list(V) if isinstance(V, (list, tuple)) else [int(V)] * self.depth
         self.R, self.n = R, n
@@ -45,7 +47,11 @@ class BeamSearch:
         ps, pn, B_in = self.parents(t)
         native.beam_step(self.trie, t, logits, ps, pn, self.R, B_in, self.n, self.V[t],
                          self.scores[t], self.bp_parent[t], self.bp_code[t], self.nodes[t],
-                         self.workspace, stream=stream)
+                         self.workspace, stream=stream, skip_rows=self.skip_rows)
+
+    def skipped_rows(self, stream=None) -> int:
+        """Rows left unread by row skipping since the last call."""
+        return native.beam_step_skipped_rows(self.workspace, stream=stream)
 
     def finalize(self, stream=None):
         native.beam_finalize(self.depth, self.R, self.n, self.bp_parent, self.bp_code,
