@@ -314,32 +314,49 @@ def measure_catalog(tcb, trie4, cat4, w4, dev):
     from sidgen import host
     from sidgen.workloads import WORKLOADS
 
-    def run(trie, n_leaves, R, L, V, K, seed, sigma, reps=50):
+    def run(trie, n_leaves, R, L, V, K, seed, sigma, reps=50, sim=None):
         table = torch.from_numpy(host.table_logits(seed, R, L, V, sigma)).to(dev).log_softmax(-1)
         table = table.contiguous()
         out_s = torch.empty((R, K), device=dev)
         out_l = torch.empty((R, K), dtype=torch.int32, device=dev)
         ws = torch.zeros(tcb.catalog_score_workspace_size(trie, R, K), dtype=torch.uint8, device=dev)
+        if sim is not None:  # (user f32 [R, d], SID embeddings bf16 bits [N, d])
+            u = torch.from_numpy(sim[0]).to(dev)
+            e = torch.from_numpy(np.ascontiguousarray(sim[1]).view(np.int16)).to(dev)
+
+            def call():
+                tcb.catalog_score_topk_sim(trie, table, u, e, R, K, out_s, out_l, ws)
+        else:
+            def call():
+                tcb.catalog_score_topk(trie, table, R, K, out_s, out_l, ws)
         for _ in range(3):
-            tcb.catalog_score_topk(trie, table, R, K, out_s, out_l, ws)
+            call()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
-            tcb.catalog_score_topk(trie, table, R, K, out_s, out_l, ws)
+            call()
         e1.record()
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / reps
         assert tcb.sidbeam_get_device_status(ws) == 0
-        return {"us_per_call": us, "pairs_per_s": R * n_leaves / (us * 1e-6),
-                "requests": R, "sids": n_leaves, "depth": L, "codes_per_level": V, "K": K}
+        out = {"us_per_call": us, "pairs_per_s": R * n_leaves / (us * 1e-6),
+               "requests": R, "sids": n_leaves, "depth": L, "codes_per_level": V, "K": K}
+        if sim is not None:
+            out["similarity_dim"] = int(sim[0].shape[1])
+        return out
 
     w2 = WORKLOADS[2]
     cat2 = w2.catalog()
     trie2 = tcb.sid_trie_build(cat2, w2.codes_per_level, w2.layouts)
     a = run(trie2, _n_leaves(cat2), w2.R, w2.depth, w2.V, w2.K, w2.logits_seed, w2.table_sigma)
+    n2 = _n_leaves(cat2)
+    sim2 = (host.user_vectors(w2.sim_seed, w2.R, w2.sim_dim, w2.user_sigma),
+            host.sid_embeddings(w2.sim_seed, n2, w2.sim_dim, w2.emb_sigma))
+    a2 = run(trie2, n2, w2.R, w2.depth, w2.V, w2.K, w2.logits_seed, w2.table_sigma, sim=sim2)
     b = run(trie4, _n_leaves(cat4), 32, w4.depth, w4.V, 10, w4.logits_seed + 7, 1.5, reps=10)
-    return {"unit": "(request, SID) pairs/s", "sprint_opq_50k": a, "wide_beam_8M_x32": b}
+    return {"unit": "(request, SID) pairs/s", "sprint_opq_50k": a,
+            "sprint_opq_50k_with_similarity": a2, "wide_beam_8M_x32": b}
 
 
 def measure_fused(tcb, dev, reps=20):

@@ -240,6 +240,24 @@ int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K
                        float* out_scores, int32_t* out_leaf, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* catalog_score_topk_sim -- catalog_score_topk plus the SID-level similarity
+ * term of the same page (inference paragraph: token log-probability sum plus
+ * SID-level similarity, then top-K; closing paragraph: one pass gives the
+ * L-by-M table and a user vector, and scoring a SID is a lookup plus one matrix
+ * product). score = sum_l logp[r][l][code_l(j)] + <user[r], sid_emb[j]>, the
+ * dot product in fp32 (four partial sums over k = 0, 1, 2, 3 mod 4, added
+ * pairwise), added after the lookup sum.
+ * The pages give no weight between the terms (a scale of user[r] is one).
+ *  user     device f32 [R][d]; sid_emb device bf16 [N][d] (N = the trie's
+ *           leaf count, row j = leaf id j as sid_trie_leaf_codes orders them),
+ *           16-byte aligned (else ALIGNMENT); d a multiple of 8 in [8, 1024].
+ *  Other arguments as catalog_score_topk (same workspace size). Errors:
+ *  INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA. */
+int catalog_score_topk_sim(const sidbeam_trie* trie, const float* logp, const float* user,
+                           const uint16_t* sid_emb, int d, int R, int K, float* out_scores,
+                           int32_t* out_leaf, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* ---------------------------------------------------------------- SID-range lm_head
  * lmhead_logits -- flashrec 0.1.0, Features > Decoding ("SID constraint"): the
  * lm_head evaluated only over the SID token range. For every row and code:

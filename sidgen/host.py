@@ -49,6 +49,8 @@ STREAM_BEAM_LOGITS = 0
 STREAM_TABLE = 1
 STREAM_HIDDEN = 2
 STREAM_WEIGHT = 3
+STREAM_USER = 4
+STREAM_SID_EMB = 5
 
 _IH_TERMS = 8            # eight 16-bit uniforms per normal draw
 _IH_MAX = 65535
@@ -210,6 +212,25 @@ def weight_matrix(seed: int, V: int, d: int, sigma: float = 0.02,
         c = np.arange(c0, min(V, c0 + chunk_rows), dtype=np.uint64)[:, None]
         x = normal_from_counters(seed, c, k, np.uint64(0), np.uint64(STREAM_WEIGHT), sigma)
         out[c0:c0 + c.shape[0]] = f32_to_bf16_bits(x)
+    return out
+
+
+def user_vectors(seed: int, R: int, d: int, sigma: float) -> np.ndarray:
+    """Per-request user vectors f32 [R, d] at counters (r, k, 0, STREAM_USER)."""
+    r = np.arange(R, dtype=np.uint64)[:, None]
+    k = np.arange(d, dtype=np.uint64)[None, :]
+    return normal_from_counters(seed, r, k, np.uint64(0), np.uint64(STREAM_USER), sigma)
+
+
+def sid_embeddings(seed: int, N: int, d: int, sigma: float, chunk_rows: int = 4096) -> np.ndarray:
+    """Per-SID embeddings, bf16 bits [N, d] (row j = leaf id j), at counters
+    (j, k, 0, STREAM_SID_EMB)."""
+    out = np.empty((N, d), dtype=np.uint16)
+    k = np.arange(d, dtype=np.uint64)[None, :]
+    for j0 in range(0, N, chunk_rows):
+        j = np.arange(j0, min(N, j0 + chunk_rows), dtype=np.uint64)[:, None]
+        x = normal_from_counters(seed, j, k, np.uint64(0), np.uint64(STREAM_SID_EMB), sigma)
+        out[j0:j0 + j.shape[0]] = f32_to_bf16_bits(x)
     return out
 
 

@@ -4,7 +4,8 @@ They stand in for the pages' workloads (RecIF-Bench / OneRec traffic, Sohu
 traffic, Amazon/Yelp catalogs), none of which is available: SID depth 3-5,
 codebooks of 256-8192 codes, beam widths 8-512 across concurrent requests,
 catalogs from thousands to millions of SIDs. Seeds: catalog 1000*c + 1,
-logits / hidden states 1000*c + 2, lm_head weight 1000*c + 3. Every request's
+logits / hidden states 1000*c + 2, lm_head weight 1000*c + 3, user and SID
+vectors of the catalog scorer's similarity term 1000*c + 4. Every request's
 prefix-hash chain starts from its own root (``host.request_roots``), so concurrent
 requests search different logits.
 """
@@ -35,6 +36,9 @@ class Workload:
     sigma: float
     K: int = 0            # catalog scorer top-K (0 = not part of the workload)
     table_sigma: float = 0.0
+    sim_dim: int = 0      # catalog scorer's SID-level similarity term (user / SID vectors)
+    user_sigma: float = 1.0
+    emb_sigma: float = 0.25
     hidden_dim: int = 0   # fused lm_head variant
     hidden_sigma: float = 1.0
     weight_sigma: float = 0.02
@@ -53,6 +57,10 @@ class Workload:
         return 1000 * self.cfg + 3
 
     @property
+    def sim_seed(self) -> int:
+        return 1000 * self.cfg + 4
+
+    @property
     def codes_per_level(self) -> List[int]:
         return [self.V] * self.depth
 
@@ -66,7 +74,7 @@ WORKLOADS = {
                 layouts=[CSR] * 3, dtype="f32", sigma=2.0),
     2: Workload("sprint-opq: 32 req x beam 32, depth 4, V=256, 50k SIDs, fp32 + top-10 scorer", 2,
                 R=32, n=32, depth=4, V=256, n_sids=50_000, dists=["uniform"] * 4,
-                layouts=None, dtype="f32", sigma=1.5, K=10, table_sigma=1.5),
+                layouts=None, dtype="f32", sigma=1.5, K=10, table_sigma=1.5, sim_dim=64),
     3: Workload("flashrec-concurrency: 64 req x beam 128, depth 3, V=8192, 1M SIDs, CSR, bf16", 3,
                 R=64, n=128, depth=3, V=8192, n_sids=1_000_000,
                 dists=[("zipf", 1.1), "uniform", "uniform"], layouts=[CSR] * 3, dtype="bf16",

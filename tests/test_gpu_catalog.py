@@ -91,3 +91,91 @@ def test_catalog_scorer_equals_exhaustive_beam(tcb):
         sids, leaf, scores = search.run(logits_for)
         assert leaf[0, :K].cpu().numpy().tolist() == gl[r].tolist()
         np.testing.assert_allclose(scores[0, :K].cpu().numpy(), gs[r], atol=3 * TOL)
+
+
+# ------------------------------------------------------------------ similarity term
+def _score_sim(tcb, trie, table, user, emb, R, K):
+    import torch
+    logp = torch.from_numpy(np.ascontiguousarray(table, dtype=np.float32)).cuda()
+    u = torch.from_numpy(np.ascontiguousarray(user, dtype=np.float32)).cuda()
+    e = torch.from_numpy(np.ascontiguousarray(emb).view(np.int16)).cuda()
+    out_s = torch.empty((R, K), device="cuda")
+    out_l = torch.empty((R, K), dtype=torch.int32, device="cuda")
+    ws = torch.zeros(tcb.catalog_score_workspace_size(trie, R, K), dtype=torch.uint8, device="cuda")
+    tcb.catalog_score_topk_sim(trie, logp, u, e, R, K, out_s, out_l, ws)
+    assert tcb.sidbeam_get_device_status(ws) == 0
+    return out_s.cpu().numpy(), out_l.cpu().numpy()
+
+
+def _sim_tol(user, emb):
+    """TOL plus the fp32 dot-product bound: d * 2^-24 * max_j sum_k |u_k e_jk|."""
+    ef = np.abs(host.bf16_bits_to_f32(emb).astype(np.float64))
+    worst = (np.abs(user.astype(np.float64)) @ ef.T).max()
+    return TOL + user.shape[1] * 2.0 ** -24 * worst
+
+
+def _check_tol(gs, gl, ref, R, K, tol):
+    for r in range(R):
+        os_ = ref["score"][r]
+        v = int(np.isfinite(os_[:K]).sum())
+        assert int(np.isfinite(gs[r]).sum()) == v
+        assert np.all(gl[r, v:] == -1)
+        np.testing.assert_allclose(gs[r, :v], os_[:v], atol=tol, rtol=0)
+        for k in range(v):
+            lo = k == 0 or os_[k - 1] - os_[k] > tol
+            hi = (not np.isfinite(os_[k + 1])) or os_[k] - os_[k + 1] > tol
+            if lo and hi:
+                assert gl[r, k] == ref["leaf"][r, k]
+
+
+def test_catalog_scorer_similarity_config2(tcb):
+    """The SPRINT-like workload (32 requests, 50,000 SIDs, top-10) with d = 64
+    user and SID vectors."""
+    w = WORKLOADS[2]
+    cat = w.catalog()
+    otrie = oracle.OracleTrie(cat, w.codes_per_level)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    table = host.table_logits(w.logits_seed, w.R, w.depth, w.V, w.table_sigma)
+    user = host.user_vectors(w.sim_seed, w.R, w.sim_dim, w.user_sigma)
+    emb = host.sid_embeddings(w.sim_seed, otrie.leaves.shape[0], w.sim_dim, w.emb_sigma)
+    gs, gl = _score_sim(tcb, gtrie, table, user, emb, w.R, w.K)
+    ref = oracle.catalog_score_topk(otrie, table, w.K + 1, user, emb)
+    plain = oracle.catalog_score_topk(otrie, table, w.K)
+    assert not np.array_equal(ref["leaf"][:, :w.K], plain["leaf"])  # the term matters here
+    _check_tol(gs, gl, ref, w.R, w.K, _sim_tol(user, emb))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_catalog_scorer_similarity_random(tcb, seed):
+    rng = np.random.default_rng(700 + seed)
+    depth = int(rng.integers(1, 4))
+    V = int(rng.choice([3, 16, 100, 256]))
+    cat = host.draw_catalog(seed, int(min(V ** depth, rng.integers(1, 5000))), [V] * depth)
+    otrie = oracle.OracleTrie(cat, [V] * depth)
+    gtrie = tcb.sid_trie_build(cat, [V] * depth, None)
+    R = int(rng.integers(1, 6))
+    K = int(rng.choice([1, 5, 64, 300]))
+    d = int(rng.choice([8, 16, 72, 256]))
+    table = host.table_logits(900 + seed, R, depth, V, 1.0)
+    user = host.user_vectors(900 + seed, R, d, float(rng.uniform(0.1, 2.0)))
+    emb = host.sid_embeddings(900 + seed, otrie.leaves.shape[0], d, float(rng.uniform(0.05, 0.5)))
+    gs, gl = _score_sim(tcb, gtrie, table, user, emb, R, K)
+    ref = oracle.catalog_score_topk(otrie, table, K + 1, user, emb)
+    _check_tol(gs, gl, ref, R, K, _sim_tol(user, emb))
+
+
+def test_catalog_scorer_similarity_argument_checks(tcb):
+    import torch
+    from trie_constrained_beam_b200 import native
+    cat = host.draw_catalog(1, 40, [8, 8])
+    gtrie = tcb.sid_trie_build(cat, [8, 8], None)
+    N = 40
+    logp = torch.zeros((1, 2, 8), device="cuda")
+    out_s = torch.empty((1, 4), device="cuda")
+    out_l = torch.empty((1, 4), dtype=torch.int32, device="cuda")
+    ws = torch.zeros(tcb.catalog_score_workspace_size(gtrie, 1, 4), dtype=torch.uint8, device="cuda")
+    u = torch.zeros((1, 12), device="cuda")                       # d % 8 != 0
+    e = torch.zeros((N, 12), dtype=torch.int16, device="cuda")
+    with pytest.raises(native.SidbeamError) as ex:
+        tcb.catalog_score_topk_sim(gtrie, logp, u, e, 1, 4, out_s, out_l, ws)
+    assert ex.value.status == native.SIDBEAM_ERR_INVALID_ARG

@@ -300,6 +300,48 @@ def test_catalog_scorer_equals_beam_search_prefix_independent():
         np.testing.assert_allclose(bs["score"][0, :K], sc["score"][r], atol=1e-12)
 
 
+def test_catalog_scorer_similarity_brute_force_tiny():
+    """Token sum plus <user, sid embedding>, written out with Python loops per
+    (request, SID); the term must change the ranking somewhere."""
+    Vs = [3, 4, 2]
+    cat = host.draw_catalog(4, 15, Vs)
+    trie = oracle.OracleTrie(cat, Vs)
+    rng = np.random.default_rng(5)
+    logp = rng.normal(0, 1, size=(3, 3, 4))
+    d = 8
+    user = host.user_vectors(77, 3, d, 1.0)
+    emb = host.sid_embeddings(77, trie.leaves.shape[0], d, 0.5)
+    ef = host.bf16_bits_to_f32(emb)
+    K = 20
+    res = oracle.catalog_score_topk(trie, logp, K, user, emb)
+    plain = oracle.catalog_score_topk(trie, logp, K)
+    changed = False
+    for r in range(3):
+        items = []
+        for j, sid in enumerate(trie.leaves.tolist()):
+            tok = sum(logp[r, lv, c] for lv, c in enumerate(sid))
+            dot = sum(float(user[r, k]) * float(ef[j, k]) for k in range(d))
+            items.append((tok + dot, j))
+        items.sort(key=lambda x: (-x[0], x[1]))
+        k = len(items)
+        assert res["leaf"][r, :k].tolist() == [j for _, j in items]
+        np.testing.assert_allclose(res["score"][r, :k], [x for x, _ in items], atol=1e-12)
+        changed |= res["leaf"][r, :k].tolist() != plain["leaf"][r, :k].tolist()
+    assert changed
+
+
+def test_catalog_scorer_zero_embeddings_is_token_only():
+    Vs = [16, 16, 16]
+    cat = host.draw_catalog(6, 500, Vs)
+    trie = oracle.OracleTrie(cat, Vs)
+    table = host.table_logits(66, 2, 3, 16, 1.5)
+    user = host.user_vectors(66, 2, 16, 1.0)
+    zero = np.zeros((trie.leaves.shape[0], 16), dtype=np.uint16)   # bf16 +0.0
+    a = oracle.catalog_score_topk(trie, table, 10, user, zero)
+    b = oracle.catalog_score_topk(trie, table, 10)
+    assert np.array_equal(a["leaf"], b["leaf"]) and np.array_equal(a["score"], b["score"])
+
+
 # ------------------------------------------------------------------ lm_head
 def test_lmhead_one_hot_picks_weight_column():
     d, V = 16, 10

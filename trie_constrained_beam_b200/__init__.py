@@ -13,6 +13,7 @@ from .native import (  # noqa: F401
     beam_step_noalloc,
     beam_step_workspace_size,
     catalog_score_topk,
+    catalog_score_topk_sim,
     catalog_score_workspace_size,
     fused_lmhead_step,
     fused_lmhead_workspace_size,

@@ -4,6 +4,13 @@
 // trie is scored by the sum of its tokens' per-position log-probabilities (a
 // lookup in an L-by-M table per request), and the K best are returned.
 //
+// With a user vector u_r per request and an embedding e_j per catalog SID the
+// score also gets the SID-level similarity term of that paragraph (and of the
+// closing paragraph: one pass gives the table and a user vector; scoring a SID
+// is a lookup plus one matrix product): score += <u_r, e_j>, the [R x d] x
+// [N x d]^T product computed pair by pair next to the lookup, in fp32 from the
+// bf16 embeddings (four interleaved partial sums, added pairwise at the end).
+//
 // (request, leaf) pairs are laid out request-major and split evenly over the
 // CTAs, exactly like beam rows in beam_step. A CTA keeps the current
 // request's table in shared memory, each warp scores 32 leaves at a time from
@@ -28,7 +35,7 @@ constexpr int kScoreWarps = 8;
 
 struct ScoreConfig {
   int W, Cw, ctas_per_sm;
-  int off_ctl, off_chist, off_whist, off_table, off_wkeys, off_wvals, smem_bytes;
+  int off_ctl, off_chist, off_whist, off_table, off_user, off_wkeys, off_wvals, smem_bytes;
 };
 
 struct ScoreArgs {
@@ -50,6 +57,10 @@ struct ScoreArgs {
   uint32_t* ghist;
   Partition part;
   ScoreConfig cfg;
+  const float* user;      // [R][d] f32, or null (no similarity term)
+  const uint16_t* emb;    // [N][d] bf16 bits, leaf-id order
+  int d;                  // multiple of 8
+  const float* emb_norm;  // max_j ||e_j||, for the histogram reference
 };
 
 struct ScoreWriter {
@@ -63,6 +74,26 @@ struct ScoreWriter {
   }
 };
 
+// max_j ||e_j||_2 of the embedding rows (one warp per row, atomicMax on the
+// bits of a non-negative float, which order like the values); *out must start
+// at zero.
+__global__ void emb_norm_kernel(const uint16_t* emb, int64_t N, int d, float* out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  float best = 0.f;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       j < N; j += warps) {
+    float s = 0.f;
+    for (int k = lane; k < d; k += 32) {
+      const float x = __uint_as_float(static_cast<uint32_t>(emb[j * d + k]) << 16);
+      s = fmaf(x, x, s);
+    }
+    best = fmaxf(best, warp_sum(s));
+  }
+  if (lane == 0) atomicMax(reinterpret_cast<unsigned*>(out), __float_as_uint(sqrtf(best)));
+}
+
+template <int SIM>
 __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     catalog_score_kernel(const __grid_constant__ ScoreArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -71,6 +102,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
   uint32_t* cta_hist = reinterpret_cast<uint32_t*>(smem + cfg.off_chist);
   uint32_t* whist = reinterpret_cast<uint32_t*>(smem + cfg.off_whist);
   float* table = reinterpret_cast<float*>(smem + cfg.off_table);
+  float* user = reinterpret_cast<float*>(smem + cfg.off_user);
   uint64_t* wkeys = reinterpret_cast<uint64_t*>(smem + cfg.off_wkeys);
   int32_t* wvals = reinterpret_cast<int32_t*>(smem + cfg.off_wvals);
 
@@ -95,6 +127,9 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     const int64_t seg_hi = min(row_hi, static_cast<int64_t>(r + 1) * a.N);
     const float* src = a.logp + static_cast<size_t>(r) * tsize;
     for (int i = threadIdx.x; i < tsize; i += blockDim.x) table[i] = src[i];
+    if (SIM)
+      for (int i = threadIdx.x; i < a.d; i += blockDim.x)
+        user[i] = a.user[static_cast<size_t>(r) * a.d + i];
     team_sync(team);
     const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
     // Histogram reference: the largest possible SID score of this request
@@ -104,6 +139,11 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
       float mx = __int_as_float(0xFF800000);
       for (int c = lane; c < a.Vmax; c += 32) mx = fmaxf(mx, table[l * a.Vmax + c]);
       C += warp_max(mx);
+    }
+    if (SIM) {  // the similarity adds at most ||u_r|| max_j ||e_j|| (Cauchy-Schwarz)
+      float uu = 0.f;
+      for (int k = lane; k < a.d; k += 32) uu = fmaf(user[k], user[k], uu);
+      C += sqrtf(warp_sum(uu)) * *a.emb_norm;
     }
     if (!(C > __int_as_float(0xFF800000) && C < __int_as_float(0x7F800000))) C = 0.f;
     const int64_t j_lo = seg_lo - static_cast<int64_t>(r) * a.N;
@@ -118,6 +158,24 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
         score = table[a.leaf_codes[j]];
         for (int l = 1; l < a.depth; ++l)
           score += table[l * a.Vmax + a.leaf_codes[static_cast<int64_t>(l) * a.stride + j]];
+        if (SIM) {  // <u_r, e_j>: 16-byte loads of the leaf's bf16 row, four partial sums
+          const uint4* er = reinterpret_cast<const uint4*>(a.emb + j * a.d);
+          float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 2
+          for (int k8 = 0; k8 < (a.d >> 3); ++k8) {
+            const uint4 q = __ldg(er + k8);
+            const float* uk = user + k8 * 8;
+            d0 = fmaf(__uint_as_float(q.x << 16), uk[0], d0);
+            d1 = fmaf(__uint_as_float(q.x & 0xFFFF0000u), uk[1], d1);
+            d2 = fmaf(__uint_as_float(q.y << 16), uk[2], d2);
+            d3 = fmaf(__uint_as_float(q.y & 0xFFFF0000u), uk[3], d3);
+            d0 = fmaf(__uint_as_float(q.z << 16), uk[4], d0);
+            d1 = fmaf(__uint_as_float(q.z & 0xFFFF0000u), uk[5], d1);
+            d2 = fmaf(__uint_as_float(q.w << 16), uk[6], d2);
+            d3 = fmaf(__uint_as_float(q.w & 0xFFFF0000u), uk[7], d3);
+          }
+          score += (d0 + d1) + (d2 + d3);
+        }
       }
       const uint64_t key = make_key(score, static_cast<uint32_t>(j));
       const bool pass = valid && key >= wb.thr;
@@ -159,7 +217,7 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-bool choose_score_config(int depth, int Vmax, int K, ScoreConfig* out) {
+bool choose_score_config(int depth, int Vmax, int K, int d, ScoreConfig* out) {
   ScoreConfig c{};
   c.W = kScoreWarps;
   static_assert(kScoreWarps * 256 >= 2 * dev::kHistBins, "rank-merge scratch lives in whist");
@@ -175,6 +233,8 @@ bool choose_score_config(int depth, int Vmax, int K, ScoreConfig* out) {
   o += c.W * 1024;
   c.off_table = o;
   o = round_up(o + depth * Vmax * 4, 128);
+  c.off_user = o;
+  o = round_up(o + d * 4, 128);
   c.off_wkeys = o;
   o += c.W * c.Cw * 8;
   c.off_wvals = o;
@@ -201,28 +261,42 @@ static int score_vmax(const sidbeam_trie* t) {
 extern "C" size_t catalog_score_workspace_size(const sidbeam_trie* trie, int R, int K) {
   if (!trie || R < 1 || K < 1 || K > SIDBEAM_MAX_BEAM) return 0;
   ScoreConfig cfg;
-  if (!choose_score_config(trie->depth, score_vmax(trie), K, &cfg)) return 0;
+  if (!choose_score_config(trie->depth, score_vmax(trie), K, 0, &cfg)) return 0;
   const Partition p = make_partition(
       R, trie->n_leaves, std::min(device_sm_count() * cfg.ctas_per_sm, kMaxSegCounts));
   return workspace_layout(R, p.maxG, K).total;
 }
 
-extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K,
-                                  float* out_scores, int32_t* out_leaf, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+// Both entry points: the token-sum scorer (user == nullptr) and the one with
+// the similarity term.
+static int catalog_score_impl(const sidbeam_trie* trie, const float* logp, const float* user,
+                              const uint16_t* emb, int d, int R, int K, float* out_scores,
+                              int32_t* out_leaf, void* workspace, size_t workspace_bytes,
+                              void* stream, const char* who) {
   if (!trie || !logp || !out_scores || !out_leaf)
-    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: NULL pointer argument");
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
   if (R < 1 || K < 1 || K > SIDBEAM_MAX_BEAM)
-    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: R=%d K=%d", R, K);
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "%s: R=%d K=%d", who, R, K);
   if (static_cast<int64_t>(R) * trie->n_leaves > (1ll << 40))
-    return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk: R * leaves too large");
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "%s: R * leaves too large", who);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return set_error(SIDBEAM_ERR_WORKSPACE, "catalog_score_topk: workspace must be 256-byte aligned");
+    return set_error(SIDBEAM_ERR_WORKSPACE, "%s: workspace must be 256-byte aligned", who);
+  const bool sim = user != nullptr;
+  if (sim) {
+    if (!emb) return set_error(SIDBEAM_ERR_INVALID_ARG, "%s: NULL sid_emb", who);
+    if (d < 8 || d > 1024 || d % 8 != 0)
+      return set_error(SIDBEAM_ERR_INVALID_ARG, "%s: d=%d must be a multiple of 8 in [8, 1024]",
+                       who, d);
+    if ((reinterpret_cast<uintptr_t>(emb) & 15u) != 0)
+      return set_error(SIDBEAM_ERR_ALIGNMENT, "%s: sid_emb must be 16-byte aligned", who);
+  }
   ScoreArgs a{};
   a.Vmax = score_vmax(trie);
-  if (!choose_score_config(trie->depth, a.Vmax, K, &a.cfg))
+  ScoreConfig base;
+  if (!choose_score_config(trie->depth, a.Vmax, K, 0, &base) ||
+      !choose_score_config(trie->depth, a.Vmax, K, sim ? d : 0, &a.cfg))
     return set_error(SIDBEAM_ERR_INVALID_ARG,
-                     "catalog_score_topk: the [depth x V] table does not fit in shared memory");
+                     "%s: the [depth x V] table does not fit in shared memory", who);
   a.leaf_codes = trie->leaf_codes;
   a.stride = trie->leaf_codes_stride;
   a.N = trie->n_leaves;
@@ -231,11 +305,15 @@ extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, i
   a.K = K;
   a.out_scores = out_scores;
   a.out_leaf = out_leaf;
+  a.user = user;
+  a.emb = emb;
+  a.d = sim ? d : 0;
+  // The partition (and so the workspace) is the token-sum scorer's, whatever d.
   a.part = make_partition(
-      R, trie->n_leaves, std::min(device_sm_count() * a.cfg.ctas_per_sm, kMaxSegCounts));
+      R, trie->n_leaves, std::min(device_sm_count() * base.ctas_per_sm, kMaxSegCounts));
   const WorkspaceLayout ws = workspace_layout(R, a.part.maxG, K);
   if (!workspace || workspace_bytes < ws.total)
-    return set_error(SIDBEAM_ERR_WORKSPACE, "catalog_score_topk: workspace of %zu bytes, need %zu",
+    return set_error(SIDBEAM_ERR_WORKSPACE, "%s: workspace of %zu bytes, need %zu", who,
                      workspace_bytes, ws.total);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.status = reinterpret_cast<uint32_t*>(w + ws.status);
@@ -245,12 +323,43 @@ extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, i
   a.part_keys = reinterpret_cast<unsigned long long*>(w + ws.part_keys);
   a.part_vals = reinterpret_cast<int32_t*>(w + ws.part_vals);
   a.ghist = reinterpret_cast<uint32_t*>(w + ws.ghist);
-  cudaError_t e = cudaFuncSetAttribute(catalog_score_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       a.cfg.smem_bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (sim) {  // max_j ||e_j|| into the status block's free bytes, for the histogram reference
+    float* norm = reinterpret_cast<float*>(w + ws.status + kEmbNormOffset);
+    a.emb_norm = norm;
+    e = cudaMemsetAsync(norm, 0, sizeof(float), st);
+    if (e != cudaSuccess) return cuda_error(e, "catalog_score_topk_sim: memset");
+    const int64_t blocks64 = std::min<int64_t>((a.N + 7) / 8, 148 * 8);
+    emb_norm_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks64, 1)), 256, 0, st>>>(
+        emb, a.N, d, norm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_error(e, "catalog_score_topk_sim: norm launch");
+  }
+  const void* fn = sim ? reinterpret_cast<const void*>(&catalog_score_kernel<1>)
+                       : reinterpret_cast<const void*>(&catalog_score_kernel<0>);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, a.cfg.smem_bytes);
   if (e != cudaSuccess) return cuda_error(e, "catalog_score_topk: cudaFuncSetAttribute");
-  catalog_score_kernel<<<a.part.grid, a.cfg.W * 32, a.cfg.smem_bytes,
-                         static_cast<cudaStream_t>(stream)>>>(a);
+  if (sim)
+    catalog_score_kernel<1><<<a.part.grid, a.cfg.W * 32, a.cfg.smem_bytes, st>>>(a);
+  else
+    catalog_score_kernel<0><<<a.part.grid, a.cfg.W * 32, a.cfg.smem_bytes, st>>>(a);
   e = cudaGetLastError();
   return e == cudaSuccess ? SIDBEAM_OK : cuda_error(e, "catalog_score_topk: launch");
+}
+
+extern "C" int catalog_score_topk(const sidbeam_trie* trie, const float* logp, int R, int K,
+                                  float* out_scores, int32_t* out_leaf, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return catalog_score_impl(trie, logp, nullptr, nullptr, 0, R, K, out_scores, out_leaf,
+                            workspace, workspace_bytes, stream, "catalog_score_topk");
+}
+
+extern "C" int catalog_score_topk_sim(const sidbeam_trie* trie, const float* logp,
+                                      const float* user, const uint16_t* sid_emb, int d, int R,
+                                      int K, float* out_scores, int32_t* out_leaf,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!user) return set_error(SIDBEAM_ERR_INVALID_ARG, "catalog_score_topk_sim: NULL user");
+  return catalog_score_impl(trie, logp, user, sid_emb, d, R, K, out_scores, out_leaf, workspace,
+                            workspace_bytes, stream, "catalog_score_topk_sim");
 }

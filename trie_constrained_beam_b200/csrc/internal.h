@@ -52,5 +52,7 @@ constexpr uint32_t kStatusTimeout = 2u;
 // Byte offset, inside the workspace's first 256-byte block (after the status
 // word), of the counter of rows beam_step did not read (row skipping).
 constexpr size_t kSkippedRowsOffset = 8;
+// ... and of max_j ||e_j|| for catalog_score_topk_sim (written each call).
+constexpr size_t kEmbNormOffset = 16;
 
 }  // namespace sidbeam

@@ -43,7 +43,7 @@ EXPORTED = (
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
     "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc", "lmhead_logits",
     "fused_lmhead_workspace_size", "sidbeam_fused_lmhead_step", "beam_step_ex",
-    "beam_step_skipped_rows",
+    "beam_step_skipped_rows", "catalog_score_topk_sim",
 )
 
 STEP_SKIP_ROWS = 1  # SIDBEAM_STEP_SKIP_ROWS
@@ -87,6 +87,7 @@ def load():
     L.catalog_score_workspace_size.argtypes = [P, I32, I32]
     L.catalog_score_workspace_size.restype = SZ
     L.catalog_score_topk.argtypes = [P, P, I32, I32, P, P, P, SZ, P]
+    L.catalog_score_topk_sim.argtypes = [P, P, P, P, I32, I32, I32, P, P, P, SZ, P]
     L.sidbeam_get_device_status.argtypes = [P, P]
     L.lmhead_logits.argtypes = [P, P, I32, I32, I32, P, I64, P, SZ, P]
     L.fused_lmhead_workspace_size.argtypes = [I32, I32, I32, I32]
@@ -100,7 +101,7 @@ def load():
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
                  "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
                  "sidbeam_get_device_status", "lmhead_logits", "sidbeam_fused_lmhead_step",
-                 "beam_step_ex", "beam_step_skipped_rows"):
+                 "beam_step_ex", "beam_step_skipped_rows", "catalog_score_topk_sim"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -258,6 +259,20 @@ def catalog_score_topk(trie, logp, R, K, out_scores, out_leaf, workspace, stream
                                    _ptr(out_leaf), _ptr(workspace),
                                    0 if workspace is None else workspace.numel() * workspace.element_size(),
                                    _stream(stream))
+    _check(rc)
+
+
+def catalog_score_topk_sim(trie, logp, user, sid_emb, R, K, out_scores, out_leaf, workspace,
+                           stream=None):
+    """catalog_score_topk plus <user[r], sid_emb[leaf]>: user f32 [R][d], sid_emb
+    bf16 [N][d] (leaf-id order), both on the device."""
+    d = int(user.shape[1])
+    if int(sid_emb.shape[1]) != d:
+        raise ValueError("user and sid_emb disagree on d")
+    rc = load().catalog_score_topk_sim(trie.handle, _ptr(logp), _ptr(user), _ptr(sid_emb), d, R,
+                                       K, _ptr(out_scores), _ptr(out_leaf), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream))
     _check(rc)
 
 
