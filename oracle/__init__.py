@@ -44,3 +44,4 @@ from .beam import (  # noqa: F401
 )
 from .catalog import catalog_score_topk  # noqa: F401
 from .lmhead import lmhead_logits, fused_lmhead_step  # noqa: F401
+from .gumbel import beam_step_gumbel, gumbel, philox4x32_10  # noqa: F401

@@ -342,6 +342,79 @@ def test_catalog_scorer_zero_embeddings_is_token_only():
     assert np.array_equal(a["leaf"], b["leaf"]) and np.array_equal(a["score"], b["score"])
 
 
+# ------------------------------------------------------------------ Gumbel top-k
+def test_oracle_philox_known_answers():
+    """The oracle's own Philox4x32-10 against the published known-answer vectors."""
+    for cols in _kat_rows():
+        v = [int(x, 16) for x in cols]
+        out = oracle.philox4x32_10(v[0], v[1], v[2], v[3], v[4], v[5])
+        assert [int(x) for x in out] == v[6:10]
+
+
+def _kat_rows():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "philox4x32_10_kat.txt")
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line.split()
+
+
+def test_gumbel_at_zero_temperature_is_deterministic_top_k():
+    Vs = [16, 16]
+    cat = host.draw_catalog(9, 120, Vs)
+    trie = oracle.OracleTrie(cat, Vs)
+    rng = np.random.default_rng(9)
+    R, B_in, n = 2, 6, 10
+    z = rng.normal(0, 2, size=(R * B_in, 16))
+    ps = np.sort(rng.uniform(-5, -1, size=R * B_in))[::-1]
+    pn = rng.integers(0, trie.n_nodes(1), size=R * B_in)
+    g = oracle.beam_step_gumbel(trie, 1, z, ps, pn, R, B_in, n, 16, 0.0, 1234)
+    d = oracle.beam_step(trie, 1, z, ps, pn, R, B_in, n, 16)
+    for k in ("score", "parent", "code", "node"):
+        assert np.array_equal(g[k], d[k])
+
+
+def _draws(z, T, n, seeds):
+    """Codes chosen, in rank order, from one root row with every code valid."""
+    V = z.shape[0]
+    out = []
+    for seed in seeds:
+        res = oracle.beam_step_gumbel(None, 0, z[None], [0.0], [0], 1, 1, n, V, T, seed)
+        out.append(tuple(res["code"][0].tolist()))
+    return out
+
+
+def test_gumbel_top1_draws_follow_tempered_softmax():
+    """The top key is a draw from softmax(log p / T): chi-square over 6,000 seeds
+    (a sign or scale error in the Gumbel transform fails it)."""
+    z = np.array([1.0, 0.2, -0.5, 0.0])
+    for T in (1.0, 0.5):
+        draws = _draws(z, T, 1, range(6000))
+        lp = oracle.log_softmax_full(z)
+        p = np.exp(lp / T)
+        p /= p.sum()
+        counts = np.bincount([d[0] for d in draws], minlength=4)
+        exp = p * len(draws)
+        chi2 = float(((counts - exp) ** 2 / exp).sum())
+        assert chi2 < 20.0, (T, counts, exp)   # 3 dof; P(chi2 > 20) < 2e-4
+
+
+def test_gumbel_top2_is_without_replacement():
+    """The ordered pair (first, second) follows p_a * p_b / (1 - p_a): the second
+    key continues the draw without the first."""
+    z = np.array([0.8, 0.0, -0.6])
+    draws = _draws(z, 1.0, 2, range(6000))
+    p = np.exp(oracle.log_softmax_full(z))
+    pairs = [(a, b) for a in range(3) for b in range(3) if a != b]
+    counts = np.array([sum(1 for d in draws if d == pr) for pr in pairs], dtype=np.float64)
+    exp = np.array([p[a] * p[b] / (1 - p[a]) for a, b in pairs]) * len(draws)
+    assert all(d[0] != d[1] for d in draws)
+    chi2 = float(((counts - exp) ** 2 / exp).sum())
+    assert chi2 < 25.0, (counts, exp)          # 5 dof; P(chi2 > 25) < 2e-4
+
+
 # ------------------------------------------------------------------ lm_head
 def test_lmhead_one_hot_picks_weight_column():
     d, V = 16, 10
