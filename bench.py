@@ -274,6 +274,9 @@ def run_ours(args, world, rank, local):
     fused = None
     if not args.no_fused:
         fused = measure_fused(tcb, dev)
+    gumbel = None
+    if not args.no_gumbel:
+        gumbel = measure_gumbel(tcb, trie, w, base, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -298,6 +301,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "catalog_score": cat_lines,
         "fused_lmhead": fused,
+        "gumbel_top_k": gumbel,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": K * (w.depth + 1),
@@ -357,6 +361,41 @@ def measure_catalog(tcb, trie4, cat4, w4, dev):
     b = run(trie4, _n_leaves(cat4), 32, w4.depth, w4.V, 10, w4.logits_seed + 7, 1.5, reps=10)
     return {"unit": "(request, SID) pairs/s", "sprint_opq_50k": a,
             "sprint_opq_50k_with_similarity": a2, "wide_beam_8M_x32": b}
+
+
+def measure_gumbel(tcb, trie, w, base, dev, reps=10):
+    """The wide-beam search with Gumbel top-k draws at temperature 1 (beam_step_gumbel)
+    on the deterministic search's logits tensors (same shapes; the drawn beams
+    differ): per-step device times from events between eager launches, and
+    logits scored per second over the whole search."""
+    import torch
+    search = tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth, temperature=1.0,
+                            seed=0x5EED_0F_6B3E1)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(w.depth + 1)]
+
+    def once(record):
+        for t in range(w.depth):
+            if record:
+                evs[t].record()
+            search.step(t, base[t])
+        if record:
+            evs[w.depth].record()
+
+    for _ in range(2):
+        once(False)
+    torch.cuda.synchronize()
+    per = np.zeros(w.depth)
+    for _ in range(reps):
+        once(True)
+        torch.cuda.synchronize()
+        per += [evs[t].elapsed_time(evs[t + 1]) * 1e3 for t in range(w.depth)]
+    per /= reps
+    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+    logits = sum(search.rows(t) * w.V for t in range(w.depth))
+    return {"temperature": 1.0, "step_us": [float(x) for x in per],
+            "logits_per_s": logits / (per.sum() * 1e-6),
+            "timing": "eager launches, events between steps, 10 searches",
+            "note": "Gumbel steps walk every row in shared memory (no register rows)"}
 
 
 def measure_fused(tcb, dev, reps=20):
@@ -552,6 +591,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused lm_head (tcgen05) lines")
+    ap.add_argument("--no-gumbel", action="store_true",
+                    help="skip the Gumbel top-k search line")
     ap.add_argument("--no-catalog", action="store_true",
                     help="skip the catalog_score_topk throughput lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -182,6 +182,30 @@ int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits, sidbeam
                  int32_t* out_code, int32_t* out_node, void* workspace, size_t workspace_bytes,
                  void* stream, unsigned flags);
 
+/* beam_step_gumbel -- beam_step at temperature > 0: Gumbel top-k without
+ * replacement (flashrec 0.1.0, Features > Serving, "API"; the second of the
+ * "next" items). Candidate c of parent slot b in request r, with the usual
+ * score x = s_b + (z_c - lse_b), is ranked by the key x + T*G, G = -log(-log U)
+ * a standard Gumbel variate: U = (v + 1/2) * 2^-23 with v the top 23 bits of
+ * the first output word of Philox4x32-10 (Salmon et al., SC'11) on the counter
+ * (r, b, c, step) with key (seed low 32 bits, seed high 32 bits). The n largest
+ * keys are kept, ranked by key (ties: parent asc, code asc), which draws n
+ * candidates without replacement in proportion to exp(x / T). The beams keep
+ * the unperturbed score: out_scores[r][i] = x of the i-th drawn candidate, so
+ * the next step adds plain log-probabilities (and out_scores are in draw
+ * order, not sorted). temperature = 0 is exactly beam_step; it must be
+ * finite and >= 0 (else INVALID_ARG).
+ *  workspace >= beam_step_gumbel_workspace_size(R, B_in, n_out, V) bytes
+ *  (beam_step's workspace plus every row's lse), zero-filled before first use.
+ *  Other arguments, results and errors: those of beam_step. Rows are walked in
+ *  shared memory (no register rows), so the step is slower than beam_step. */
+size_t beam_step_gumbel_workspace_size(int R, int B_in, int n_out, int V);
+int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dtype dtype,
+                     int64_t ld, const float* parent_scores, const int32_t* parent_nodes, int R,
+                     int B_in, int n_out, int V, float temperature, uint64_t seed,
+                     float* out_scores, int32_t* out_parent, int32_t* out_code,
+                     int32_t* out_node, void* workspace, size_t workspace_bytes, void* stream);
+
 /* beam_step_skipped_rows -- rows not read by row skipping since the last call
  * on this workspace (host *count); the counter is reset to zero. `stream`
  * orders the read after the steps that used the workspace (the call

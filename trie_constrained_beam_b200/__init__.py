@@ -9,6 +9,8 @@ from .native import (  # noqa: F401
     Trie,
     beam_finalize,
     beam_step,
+    beam_step_gumbel,
+    beam_step_gumbel_workspace_size,
     beam_step_skipped_rows,
     beam_step_noalloc,
     beam_step_workspace_size,

@@ -39,7 +39,8 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      const float* parent_scores, const int32_t* parent_nodes, int R, int B_in,
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream, unsigned flags);
+                     cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
+                     float* row_lse);
 
 namespace {
 
@@ -106,7 +107,7 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
                             float* out_scores, int32_t* out_parent, int32_t* out_code,
                             int32_t* out_node, void* workspace, size_t workspace_bytes,
                             void* stream, unsigned flags) {
-  if (flags & ~static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS))
+  if (flags & ~(static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS) | kValidateOnly))
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
   if (!logits || !parent_scores || !out_scores || !out_parent || !out_code || !out_node)
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: NULL pointer argument");
@@ -142,9 +143,51 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
   }
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step: workspace must be 256-byte aligned");
+  if (flags & kValidateOnly) return SIDBEAM_OK;
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
-                          workspace_bytes, static_cast<cudaStream_t>(stream), flags);
+                          workspace_bytes, static_cast<cudaStream_t>(stream), flags, 0.f, 0ull,
+                          nullptr);
+}
+
+// Gumbel steps keep every row's lse after the beam_step workspace.
+static size_t gumbel_lse_offset(int R, int B_in, int n_out, int V) {
+  return (beam_step_workspace_size(R, B_in, n_out, V) + 255) & ~static_cast<size_t>(255);
+}
+
+extern "C" size_t beam_step_gumbel_workspace_size(int R, int B_in, int n_out, int V) {
+  const size_t base = beam_step_workspace_size(R, B_in, n_out, V);
+  if (base == 0) return 0;
+  return gumbel_lse_offset(R, B_in, n_out, V) + static_cast<size_t>(R) * B_in * sizeof(float);
+}
+
+extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* logits,
+                                sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                                const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                                float temperature, uint64_t seed, float* out_scores,
+                                int32_t* out_parent, int32_t* out_code, int32_t* out_node,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!(temperature >= 0.f) || temperature > 1e30f)
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step_gumbel: temperature must be finite, >= 0");
+  if (temperature == 0.f)  // the deterministic step
+    return beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
+                        n_out, V, out_scores, out_parent, out_code, out_node, workspace,
+                        workspace_bytes, stream, 0u);
+  const size_t need = beam_step_gumbel_workspace_size(R, B_in, n_out, V);
+  if (need == 0 || workspace_bytes < need)
+    return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step_gumbel: workspace of %zu bytes, need %zu",
+                     workspace_bytes, need);
+  // The shape checks of beam_step, then the Gumbel launch.
+  const int rc = beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
+                              n_out, V, out_scores, out_parent, out_code, out_node, nullptr, 0,
+                              stream, kValidateOnly);
+  if (rc != SIDBEAM_OK) return rc;
+  float* row_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                            gumbel_lse_offset(R, B_in, n_out, V));
+  return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
+                          n_out, V, out_scores, out_parent, out_code, out_node, workspace,
+                          workspace_bytes, static_cast<cudaStream_t>(stream), 0u, temperature,
+                          seed, row_lse);
 }
 
 extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,

@@ -100,6 +100,90 @@ struct StepArgs {
   int coop;  // 1: every warp takes every row of the CTA (fewer rows than warps)
   int skip_rows;     // 1: rows whose parent score is below the request's bound are not read
   uint32_t* skipped; // counter of rows not read for that reason
+  // Gumbel top-k (temperature gumbel_T > 0; the kernel instantiation with GUM = 1)
+  float gumbel_T;
+  uint32_t gseed0, gseed1;  // Philox key (seed lo, hi)
+  int gstep;                // counter word 3
+  float* row_lse;           // [R * B_in]: every live row's lse (the writer needs it)
+};
+
+// ------------------------------------------------------------ Gumbel top-k
+// Temperature T > 0 (flashrec 0.1.0, Features > Serving, "API": Gumbel top-k
+// without replacement above temperature 0): candidate c of parent slot b in
+// request r gets the key of s + (z_c + T*G - lse), G a standard Gumbel
+// variate for (r, b, c, step); the n largest keys are a draw of n candidates
+// without replacement in proportion to exp(score / T), and the beams keep
+// the unperturbed score (written out from the row's logits and lse).
+// G = -log(-log U), U = (v + 1/2) 2^-23 exact in fp32, v = the top 23 bits of
+// the first word of Philox4x32-10 (Salmon et al., SC'11) on counter
+// (r, b, c, step), key = the seed. G <= kGumbelMax for every U.
+constexpr float kGumbelMax = 16.7f;
+
+__device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                 uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    if (i > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return c0;
+}
+
+// T * G for candidate (r, b, code).
+__device__ __forceinline__ float gumbel_noise(const StepArgs& a, int r, uint32_t b, int code) {
+  const uint32_t v = philox_word0(static_cast<uint32_t>(r), b, static_cast<uint32_t>(code),
+                                  static_cast<uint32_t>(a.gstep), a.gseed0, a.gseed1) >> 9;
+  const float U = (static_cast<float>(v) + 0.5f) * 1.1920928955078125e-07f;  // 2^-23
+  return a.gumbel_T * -logf(-logf(U));
+}
+
+// The writer of a Gumbel step: the ranks follow the perturbed keys; the score
+// written is the unperturbed s + (z - lse), recomputed from the row exactly as
+// the deterministic step computes it.
+struct GumbelWriter {
+  float* scores;
+  int32_t* parent;
+  int32_t* code;
+  int32_t* node;
+  int n;
+  uint32_t V;
+  const uint8_t* logits;
+  int64_t row_bytes;
+  int bf16;
+  const float* parent_scores;
+  const float* row_lse;
+  int B_in;
+  __device__ __forceinline__ void operator()(int r, int i, uint64_t key, int32_t val,
+                                             bool valid) const {
+    const size_t o = static_cast<size_t>(r) * n + i;
+    if (valid) {
+      const uint32_t idx = key_idx(key);
+      const int32_t b = static_cast<int32_t>(idx / V), c = static_cast<int32_t>(idx % V);
+      const int64_t row = static_cast<int64_t>(r) * B_in + b;
+      const uint8_t* zr = logits + row * row_bytes;
+      const float z = bf16 ? __uint_as_float(static_cast<uint32_t>(
+                                 reinterpret_cast<const uint16_t*>(zr)[c]) << 16)
+                           : reinterpret_cast<const float*>(zr)[c];
+      scores[o] = parent_scores[row] + (z - row_lse[row]);
+      parent[o] = b;
+      code[o] = c;
+      node[o] = val;
+    } else {
+      scores[o] = __int_as_float(0xFF800000);
+      parent[o] = -1;
+      code[o] = -1;
+      node[o] = -1;
+    }
+  }
 };
 
 struct StepWriter {
@@ -543,6 +627,8 @@ struct RowCtx {
   uint32_t idx0;  // b * V (key index of code 0)
   uint32_t o0;    // first child id
   uint32_t o1;    // one past the last child id
+  int r;          // request (Gumbel counters)
+  uint32_t b;     // parent slot in the request
 };
 
 // Code of CSR child id k: from the stage when it was staged, else from HBM/L2.
@@ -756,13 +842,21 @@ __device__ __noinline__ uint64_t push_histogram(const StepArgs& a, SelCtl* ctl, 
                                                 uint64_t thr, ThrSinks sinks, int lane);
 // r: the row's request; multi: the request is split over several CTAs (the
 // count pass then also pushes, so that the offer pass sees their counts).
-template <int BF16>
+// GUM: Gumbel top-k (see gumbel_noise): every candidate's logit is replaced
+// by z + T*G before its key is formed, and the bulk tests (row max, vector
+// max) allow for the largest possible T*G.
+template <int BF16, int GUM = 0>
 __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& c, float rmax,
                           float zthr, WarpBuf& wb, SelCtl* ctl, uint32_t* wprefix,
                           uint32_t* wmask, const ThrSinks& sinks, int lane, int part,
                           int nparts, int r, bool multi) {
   constexpr int kPerVec = BF16 ? 8 : 4;
-  if (rmax < zthr) return;  // even the row's largest logit cannot reach the threshold
+  const float gm = GUM ? a.gumbel_T * kGumbelMax : 0.f;  // bound on T*G
+  auto zeff = [&](float z, int code) -> float {
+    if constexpr (GUM) return z + gumbel_noise(a, c.r, c.b, code);
+    return z;
+  };
+  if (rmax + gm < zthr) return;  // even the row's largest logit cannot reach the threshold
   const uint32_t* mrow = nullptr;  // valid-child bitmap (null: every code is valid)
   int words = 0;
   if (a.layout == SIDBEAM_LAYOUT_CSR) {
@@ -773,7 +867,7 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
         const uint32_t k = k0 + lane;
         const bool in = k < c.o1;
         const int code = in ? csr_code(a, zrow, c.o0, nst, k) : 0;
-        const float z = in ? elem<BF16>(zrow, code) : 0.f;
+        const float z = in ? zeff(elem<BF16>(zrow, code), code) : 0.f;
         const bool ok = in && z >= zthr;
         if (!__any_sync(kFull, ok)) continue;
         const float score = c.s + (z - c.lse);
@@ -801,21 +895,33 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
     for (int v0 = part * 32; v0 < nvec_all; v0 += 32 * nparts) {
       const int v = v0 + lane;
       unsigned bits = 0u;
+      float zp[kPerVec];  // effective logits of the hits (GUM)
       const uint4 x = v < nvec_all ? q[v] : make_uint4(0u, 0u, 0u, 0u);
-      if (v < nvec_all && vec_max<BF16>(x) >= zthr) {
+      if (v < nvec_all && vec_max<BF16>(x) + gm >= zthr) {
         const int cb = v * kPerVec;
         unsigned valid = (1u << kPerVec) - 1u;
         if (mrow) valid = (mrow[cb >> 5] >> (cb & 31)) & ((1u << kPerVec) - 1u);
         if (a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
 #pragma unroll
-        for (int j = 0; j < kPerVec; ++j)
-          if (((valid >> j) & 1u) && vec_elem<BF16>(x, j) >= zthr) bits |= 1u << j;
+        for (int j = 0; j < kPerVec; ++j) {
+          if constexpr (GUM) {
+            zp[j] = 0.f;
+            if (((valid >> j) & 1u) && vec_elem<BF16>(x, j) + gm >= zthr) {
+              zp[j] = zeff(vec_elem<BF16>(x, j), cb + j);
+              if (zp[j] >= zthr) bits |= 1u << j;
+            }
+          } else {
+            if (((valid >> j) & 1u) && vec_elem<BF16>(x, j) >= zthr) bits |= 1u << j;
+          }
+        }
       }
       if (pass == 0) {  // count the hits of this vector in one go
 #pragma unroll
         for (int j = 0; j < kPerVec; ++j)
-          if ((bits >> j) & 1u)
-            atomicAdd(&ctl->hist[score_bin(c.s + (vec_elem<BF16>(x, j) - c.lse), c.C)], 1u);
+          if ((bits >> j) & 1u) {
+            const float z = GUM ? zp[j] : vec_elem<BF16>(x, j);
+            atomicAdd(&ctl->hist[score_bin(c.s + (z - c.lse), c.C)], 1u);
+          }
         const int cnt = static_cast<int>(__reduce_add_sync(kFull, __popc(bits)));
         wb.binned += cnt;
         if (lane == 0 && cnt) atomicAdd(&ctl->hist_total, static_cast<unsigned>(cnt));
@@ -829,7 +935,7 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
       while (__any_sync(kFull, bits != 0u)) {
         const int j = bits ? __ffs(bits) - 1 : 0;
         const int code = v * kPerVec + j;
-        const float z = vec_elem<BF16>(x, j);
+        const float z = (GUM && bits) ? zeff(vec_elem<BF16>(x, j), code) : vec_elem<BF16>(x, j);
         const bool has = bits != 0u && z >= zthr;
         bits &= bits - 1u;
         const float score = c.s + (z - c.lse);
@@ -935,6 +1041,7 @@ __device__ __forceinline__ float segment_ref(const StepArgs& a, const Team& t, S
 // Once per segment, out of line (away from the per-row loop). The warp buffer
 // goes in by value so that the caller's copy stays in registers; the caller
 // empties its own copy afterwards.
+template <int GUM>
 __device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf wb, SelCtl* ctl,
                                          uint64_t* wkeys, int32_t* wvals, uint32_t* whist,
                                          uint32_t* cta_hist, uint8_t* stages, int direct_cap,
@@ -969,9 +1076,16 @@ __device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf w
   f.direct_vals =
       last ? reinterpret_cast<int32_t*>(stages + static_cast<size_t>(direct_cap) * 8) : nullptr;
   f.direct_cap = last ? direct_cap : 0;
-  const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
-                          static_cast<uint32_t>(a.V)};
-  return segment_flush(team, wb, ctl, f, writer);
+  if constexpr (GUM) {
+    const GumbelWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
+                              static_cast<uint32_t>(a.V), a.logits, a.row_bytes, a.bf16,
+                              a.parent_scores, a.row_lse, a.B_in};
+    return segment_flush(team, wb, ctl, f, writer);
+  } else {
+    const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
+                            static_cast<uint32_t>(a.V)};
+    return segment_flush(team, wb, ctl, f, writer);
+  }
 }
 
 // --------------------------------------------------------------- threshold seeding
@@ -1015,9 +1129,10 @@ __device__ void seed_count(const StepArgs& a, const uint8_t* zrow, float s, floa
 }
 
 // --------------------------------------------------------------- kernel
-template <int BF16, int REG>
+template <int BF16, int REG, int GUM = 0>
 __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 32, 1)
     beam_step_kernel(const __grid_constant__ StepArgs a) {
+  static_assert(!(REG && GUM), "Gumbel steps walk their rows in shared memory");
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kPerVec = BF16 ? 8 : 4;
   const StepConfig& cfg = a.cfg;
@@ -1152,12 +1267,13 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     }
   }
   float C = segment_ref_finish(team, ctl, ref_slot, mref);
+  if constexpr (GUM) C += a.gumbel_T * kGumbelMax;  // perturbed scores reach this high
   if (shared_rows) q = cq;  // sequence entries are CTA entries from here on
 
   // 3b. Threshold seeding from the first row of every warp that belongs to
   //     the first request, when those rows have more than n children in all
   //     (read from the shared table).
-  if (shared_rows) {
+  if (shared_rows && !GUM) {  // (Gumbel keys are not bounded by these counts)
     const int64_t end_first = static_cast<int64_t>(r_first + 1) * a.B_in;  // rows of r_first
     const int nfirst = cq.count < W ? cq.count : W;
     uint32_t nch = 0u;
@@ -1197,7 +1313,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   int req_pref_r = -1;
   // Row skipping needs a bound of the rows' own request: CTAs that hold rows
   // of one request only.
-  const bool skipping = a.skip_rows && a.part.grouped;
+  const bool skipping = !GUM && a.skip_rows && a.part.grouped;
   auto refill = [&]() {
     uint64_t bound = 0ull;
     if (skipping) {
@@ -1213,12 +1329,14 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   // End of the segment of request cur_r (all warps, in the same order).
   int cur_r = r_first;
   auto flush = [&]() -> bool {
-    const bool stop = segment_end(a, team, wb, ctl, wkeys, wvals, whist, cta_hist, stages,
+    const bool stop = segment_end<GUM>(a, team, wb, ctl, wkeys, wvals, whist, cta_hist, stages,
                                   direct_cap, cur_r, r_last, C);
     wb.count = 0;
     wb.thr = 0ull;
     if (stop) return true;
-    if (cur_r < r_last) C = segment_ref(a, team, ctl, cur_r + 1, ref_slot ^= 1);
+    if (cur_r < r_last)
+      C = segment_ref(a, team, ctl, cur_r + 1, ref_slot ^= 1) +
+          (GUM ? a.gumbel_T * kGumbelMax : 0.f);
     ++cur_r;
     return false;
   };
@@ -1249,7 +1367,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
 
     const uint32_t b = static_cast<uint32_t>(row - static_cast<int64_t>(r) * a.B_in);
     const bool multi = a.part.contributors(r) > 1;
-    RowCtx c{s, 0.f, C, b * static_cast<uint32_t>(a.V), o0, o1};
+    RowCtx c{s, 0.f, C, b * static_cast<uint32_t>(a.V), o0, o1, r, b};
     const ThrSinks sinks{&ctl->cta_thr, a.request_thr + r};
     const unsigned long long req_now = req_pref_r == r ? req_pref : 0ull;
     const bool csr = a.layout == SIDBEAM_LAYOUT_CSR;
@@ -1344,8 +1462,9 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     } else {
       float rmax;
       row_stats<BF16>(zrow, a.V, lane, rmax, c.lse);
+      if (GUM && lane == 0) a.row_lse[row] = c.lse;  // the writer recomputes scores from it
       row_thresholds(wb, ctl, req_now);
-      smem_walk<BF16>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
+      smem_walk<BF16, GUM>(a, zrow, c, rmax, zthreshold(wb.thr, c.s, c.lse), wb, ctl, my_prefix,
                       my_mask, sinks, lane, part, nparts, r, multi);
       __syncwarp();
       refresh_row(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
@@ -1451,7 +1570,7 @@ bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int
 // follows a first eager call).
 static cudaError_t opt_in_smem(const void* fn, int which) {
   static std::mutex mu;
-  static bool done[4][64] = {};
+  static bool done[6][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1468,7 +1587,8 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      const float* parent_scores, const int32_t* parent_nodes, int R, int B_in,
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
-                     cudaStream_t stream, unsigned flags) {
+                     cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
+                     float* row_lse) {
   StepArgs a{};
   a.logits = static_cast<const uint8_t*>(logits);
   a.bf16 = dtype == SIDBEAM_BF16;
@@ -1504,6 +1624,12 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   a.status = reinterpret_cast<uint32_t*>(w + ws.status);
   a.skipped = reinterpret_cast<uint32_t*>(w + ws.status + kSkippedRowsOffset);
   a.skip_rows = (flags & SIDBEAM_STEP_SKIP_ROWS) ? 1 : 0;
+  const bool gum = gumbel_T > 0.f;
+  a.gumbel_T = gum ? gumbel_T : 0.f;
+  a.gseed0 = static_cast<uint32_t>(gumbel_seed);
+  a.gseed1 = static_cast<uint32_t>(gumbel_seed >> 32);
+  a.gstep = step;
+  a.row_lse = row_lse;
   a.tickets = reinterpret_cast<uint32_t*>(w + ws.tickets);
   a.request_thr = reinterpret_cast<unsigned long long*>(w + ws.request_thr);
   a.part_count = reinterpret_cast<uint32_t*>(w + ws.part_count);
@@ -1517,7 +1643,8 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   // children (turned into a bitmap).
   const int prefix_words = dense ? a.mask_stride
                                  : (a.layout == SIDBEAM_LAYOUT_CSR ? ((V + 31) / 32 + 3) / 4 * 4 : 0);
-  const bool reg = static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
+  // (Gumbel steps walk every row in shared memory.)
+  const bool reg = !gum && static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
   if (!choose_step_config(V, esize, extra, prefix_words, n_out, reg, &a.cfg) &&
       !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, &a.cfg)))
     return set_error(SIDBEAM_ERR_INVALID_ARG,
@@ -1526,11 +1653,13 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: internal warp plan out of range");
   a.coop = a.part.rows_per_cta < a.cfg.W ? 1 : 0;
 
-  const void* fns[4] = {reinterpret_cast<const void*>(&beam_step_kernel<0, 0>),
+  const void* fns[6] = {reinterpret_cast<const void*>(&beam_step_kernel<0, 0>),
                         reinterpret_cast<const void*>(&beam_step_kernel<1, 0>),
                         reinterpret_cast<const void*>(&beam_step_kernel<0, 1>),
-                        reinterpret_cast<const void*>(&beam_step_kernel<1, 1>)};
-  const int which = (a.cfg.reg ? 2 : 0) + (a.bf16 ? 1 : 0);
+                        reinterpret_cast<const void*>(&beam_step_kernel<1, 1>),
+                        reinterpret_cast<const void*>(&beam_step_kernel<0, 0, 1>),
+                        reinterpret_cast<const void*>(&beam_step_kernel<1, 0, 1>)};
+  const int which = (gum ? 4 : (a.cfg.reg ? 2 : 0)) + (a.bf16 ? 1 : 0);
   cudaError_t e = opt_in_smem(fns[which], which);
   if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaFuncSetAttribute");
   const dim3 grid(static_cast<unsigned>(a.part.grid));
@@ -1539,7 +1668,9 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
     case 0: beam_step_kernel<0, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 1: beam_step_kernel<1, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 2: beam_step_kernel<0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    default: beam_step_kernel<1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    case 3: beam_step_kernel<1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    case 4: beam_step_kernel<0, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    default: beam_step_kernel<1, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "beam_step: launch");

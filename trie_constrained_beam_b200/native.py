@@ -43,7 +43,8 @@ EXPORTED = (
     "catalog_score_workspace_size", "catalog_score_topk", "sidbeam_get_device_status",
     "sidbeam_last_error", "sidbeam_version", "beam_step_noalloc", "lmhead_logits",
     "fused_lmhead_workspace_size", "sidbeam_fused_lmhead_step", "beam_step_ex",
-    "beam_step_skipped_rows", "catalog_score_topk_sim",
+    "beam_step_skipped_rows", "catalog_score_topk_sim", "beam_step_gumbel",
+    "beam_step_gumbel_workspace_size",
 )
 
 STEP_SKIP_ROWS = 1  # SIDBEAM_STEP_SKIP_ROWS
@@ -83,6 +84,10 @@ def load():
     L.beam_step_ex.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P,
                                ctypes.c_uint]
     L.beam_step_skipped_rows.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
+    L.beam_step_gumbel_workspace_size.argtypes = [I32, I32, I32, I32]
+    L.beam_step_gumbel_workspace_size.restype = SZ
+    L.beam_step_gumbel.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, ctypes.c_float,
+                                   ctypes.c_uint64, P, P, P, P, P, SZ, P]
     L.beam_finalize.argtypes = [I32, I32, I32, P, P, P, P, P, P]
     L.catalog_score_workspace_size.argtypes = [P, I32, I32]
     L.catalog_score_workspace_size.restype = SZ
@@ -101,7 +106,8 @@ def load():
     for name in ("sid_trie_build", "sid_trie_info", "sid_trie_leaf_rows", "sid_trie_leaf_codes",
                  "beam_step", "beam_step_noalloc", "beam_finalize", "catalog_score_topk",
                  "sidbeam_get_device_status", "lmhead_logits", "sidbeam_fused_lmhead_step",
-                 "beam_step_ex", "beam_step_skipped_rows", "catalog_score_topk_sim"):
+                 "beam_step_ex", "beam_step_skipped_rows", "catalog_score_topk_sim",
+                 "beam_step_gumbel"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -221,6 +227,27 @@ def beam_step(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V
         rc = load().beam_step_ex(*args, STEP_SKIP_ROWS)
     else:
         rc = load().beam_step(*args)
+    _check(rc)
+
+
+def beam_step_gumbel_workspace_size(R: int, B_in: int, n_out: int, V: int) -> int:
+    return int(load().beam_step_gumbel_workspace_size(R, B_in, n_out, V))
+
+
+def beam_step_gumbel(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V,
+                     temperature, seed, out_scores, out_parent, out_code, out_node, workspace,
+                     stream=None, ld=None):
+    """Gumbel top-k step at `temperature` (0: the deterministic step); `seed`
+    keys the Philox stream. Outputs in draw order; scores unperturbed."""
+    if ld is None:
+        ld = logits.stride(0)
+    rc = load().beam_step_gumbel(None if trie is None else trie.handle, step, _ptr(logits),
+                                 _dtype_code(logits), ld, _ptr(parent_scores),
+                                 _ptr(parent_nodes), R, B_in, n_out, V, float(temperature),
+                                 int(seed) & 0xFFFFFFFFFFFFFFFF, _ptr(out_scores),
+                                 _ptr(out_parent), _ptr(out_code), _ptr(out_node),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
     _check(rc)
 
 

@@ -14,9 +14,11 @@ from . import native
 
 class BeamSearch:
     def __init__(self, trie, R: int, n: int, V, depth: int = None, device="cuda",
-                 skip_rows: bool = False):
+                 skip_rows: bool = False, temperature: float = 0.0, seed: int = 0):
         self.trie = trie
         self.skip_rows = skip_rows  # beam_step_ex row skipping (same results)
+        # temperature > 0: Gumbel top-k draws (beam_step_gumbel), Philox key `seed`
+        self.temperature, self.seed = float(temperature), int(seed)
         self.depth = depth if depth is not None else trie.depth
         self.V = list(V) if isinstance(V, (list, tuple)) else [int(V)] * self.depth
         self.R, self.n = R, n
@@ -29,7 +31,9 @@ class BeamSearch:
         self.bp_code = torch.empty((self.depth, R, n), dtype=torch.int32, device=dev)
         ws = 0
         for t in range(self.depth):
-            ws = max(ws, native.beam_step_workspace_size(R, 1 if t == 0 else n, n, self.V[t]))
+            size = (native.beam_step_gumbel_workspace_size if self.temperature > 0
+                    else native.beam_step_workspace_size)
+            ws = max(ws, size(R, 1 if t == 0 else n, n, self.V[t]))
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=dev)
         self.sids = torch.empty((R, n, self.depth), dtype=torch.int32, device=dev)
         self.leaf = torch.empty((R, n), dtype=torch.int32, device=dev)
@@ -45,6 +49,12 @@ class BeamSearch:
 
     def step(self, t: int, logits, stream=None):
         ps, pn, B_in = self.parents(t)
+        if self.temperature > 0:
+            native.beam_step_gumbel(self.trie, t, logits, ps, pn, self.R, B_in, self.n,
+                                    self.V[t], self.temperature, self.seed, self.scores[t],
+                                    self.bp_parent[t], self.bp_code[t], self.nodes[t],
+                                    self.workspace, stream=stream)
+            return
         native.beam_step(self.trie, t, logits, ps, pn, self.R, B_in, self.n, self.V[t],
                          self.scores[t], self.bp_parent[t], self.bp_code[t], self.nodes[t],
                          self.workspace, stream=stream, skip_rows=self.skip_rows)
