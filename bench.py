@@ -277,6 +277,9 @@ def run_ours(args, world, rank, local):
     gumbel = None
     if not args.no_gumbel:
         gumbel = measure_gumbel(tcb, trie, w, base, dev)
+    widths = None
+    if not args.no_widths:
+        widths = measure_widths(tcb, trie, w, base, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -302,6 +305,7 @@ def run_ours(args, world, rank, local):
         "catalog_score": cat_lines,
         "fused_lmhead": fused,
         "gumbel_top_k": gumbel,
+        "per_request_widths": widths,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": K * (w.depth + 1),
@@ -396,6 +400,36 @@ def measure_gumbel(tcb, trie, w, base, dev, reps=10):
             "logits_per_s": logits / (per.sum() * 1e-6),
             "timing": "eager launches, events between steps, 10 searches",
             "note": "Gumbel steps walk every row in shared memory (no register rows)"}
+
+
+def measure_widths(tcb, trie, w, base, dev, reps=50):
+    """The wide-beam search with per-request widths 512, 384, 256, 128 (cycling
+    over the 16 requests) in one launch per step, the whole search (5 steps +
+    finalize) replayed as one CUDA graph on the deterministic search's logits;
+    slots past a request's width are dead rows of the next step (not read)."""
+    import torch
+    widths = [(512, 384, 256, 128)[r % 4] for r in range(w.R)]
+    search = tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth, widths=widths)
+    for t in range(w.depth):
+        search.step(t, base[t])
+    search.finalize()
+    torch.cuda.synchronize()
+    g = search.capture(base)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+    live = w.R * w.V + sum(widths) * w.V * (w.depth - 1)   # rows scored: roots + kept beams
+    return {"widths": "512/384/256/128 cycling over 16 requests", "us_per_search": us,
+            "logits_per_s": live / (us * 1e-6),
+            "timing": "CUDA graph of the whole search (5 beam_step + beam_finalize), 50 replays"}
 
 
 def measure_fused(tcb, dev, reps=20):
@@ -591,6 +625,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused lm_head (tcgen05) lines")
+    ap.add_argument("--no-widths", action="store_true",
+                    help="skip the per-request widths line")
     ap.add_argument("--no-gumbel", action="store_true",
                     help="skip the Gumbel top-k search line")
     ap.add_argument("--no-catalog", action="store_true",

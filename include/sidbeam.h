@@ -173,14 +173,21 @@ int beam_step(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dt
  *  each hold only that request (R no larger than the GPU's SM count); the
  *  first rows of each CTA are always read. The number of rows passed over
  *  accumulates in the workspace (beam_step_skipped_rows).
+ *  out_width: NULL, or device i32 [R] with 0 <= out_width[r] <= n_out: request r
+ *  keeps only its out_width[r] best beams; output slots past that are padding
+ *  (score -inf, indices -1), so they are dead rows of the next step and are
+ *  never read. The kept beams are exactly the first out_width[r] ranks of the
+ *  request's top n_out, the same as a step with n_out = out_width[r]: per-request
+ *  beam widths in one launch (and so in one captured graph of the whole search;
+ *  the third of the "next" items). Values outside [0, n_out] are undefined.
  *  Other arguments, results and errors: those of beam_step; unknown flag bits
- *  give INVALID_ARG. beam_step(...) is beam_step_ex(..., 0). */
+ *  give INVALID_ARG. beam_step(...) is beam_step_ex(..., 0, NULL). */
 #define SIDBEAM_STEP_SKIP_ROWS 1u
 int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dtype dtype,
                  int64_t ld, const float* parent_scores, const int32_t* parent_nodes, int R,
                  int B_in, int n_out, int V, float* out_scores, int32_t* out_parent,
                  int32_t* out_code, int32_t* out_node, void* workspace, size_t workspace_bytes,
-                 void* stream, unsigned flags);
+                 void* stream, unsigned flags, const int32_t* out_width);
 
 /* beam_step_gumbel -- beam_step at temperature > 0: Gumbel top-k without
  * replacement (flashrec 0.1.0, Features > Serving, "API"; the second of the

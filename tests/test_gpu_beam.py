@@ -431,3 +431,60 @@ def test_error_conventions(tcb):
     assert tcb.sidbeam_get_device_status(ws) == -7
     assert tcb.sidbeam_get_device_status(ws) == 0
     assert _host(o[1]).tolist()[0] == 0    # row 0 (node (0,)) still expanded
+
+
+# ---------------------------------------------------------------- per-request widths
+def _search_roots(tcb, gtrie, roots, n, depth, V, seed, sigma, widths=None, graph=False):
+    """A whole search from the given per-request root hashes (device generator
+    logits); returns (sids, leaf, scores) on the host. graph: replay a captured
+    graph of the search instead of the eager calls."""
+    import torch
+    from sidgen import device as gdev
+    R = roots.shape[0]
+    search = tcb.BeamSearch(gtrie, R, n, V, depth=depth, widths=widths)
+    hashes = torch.from_numpy(roots.view(np.int64)).to("cuda")
+    logits = []
+    for t in range(depth):
+        lg = torch.empty((search.rows(t), V), dtype=torch.float32, device="cuda")
+        gdev.row_logits(seed, hashes, V, sigma, lg)
+        search.step(t, lg)
+        assert tcb.sidbeam_get_device_status(search.workspace) == 0
+        ps, pn, B_in = search.parents(t)
+        child = torch.empty((R * n,), dtype=torch.int64, device="cuda")
+        gdev.child_hash(hashes, R, B_in, search.bp_parent[t], search.bp_code[t], n, t + 1, child)
+        hashes = child
+        logits.append(lg)
+    sids, leaf, scores = search.finalize()
+    out = [x.cpu().numpy().copy() for x in (sids, leaf, scores)]
+    if graph:
+        for x in (search.scores, search.sids):
+            x.fill_(0)
+        g = search.capture(logits)
+        g.replay()
+        torch.cuda.synchronize()
+        again = [x.cpu().numpy() for x in (search.sids, search.leaf,
+                                          search.scores[depth - 1].view(R, n))]
+        for a, b in zip(out, again):
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    return out
+
+
+def test_per_request_widths_equal_separate_searches(tcb):
+    """Four requests of widths 64, 17, 1 and 40 in one launch per step (and one
+    captured graph) give, request by request, bit for bit what a search of that
+    request alone at its own width gives; the slots past a width are padding."""
+    w = WORKLOADS[2]
+    cat, _ = _catalog(2)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    widths = [64, 17, 1, 40]
+    n = max(widths)
+    roots = host.request_roots(len(widths))
+    sids, leaf, scores = _search_roots(tcb, gtrie, roots, n, w.depth, w.V, w.logits_seed,
+                                       w.sigma, widths=widths, graph=True)
+    for r, wr in enumerate(widths):
+        s1, l1, c1 = _search_roots(tcb, gtrie, roots[r:r + 1], wr, w.depth, w.V, w.logits_seed,
+                                   w.sigma)
+        assert np.array_equal(sids[r, :wr], s1[0]) and np.array_equal(leaf[r, :wr], l1[0])
+        assert np.array_equal(scores[r, :wr].view(np.uint32), c1[0].view(np.uint32))
+        assert np.all(leaf[r, wr:] == -1) and np.all(sids[r, wr:] == -1)
+        assert np.all(np.isneginf(scores[r, wr:]))

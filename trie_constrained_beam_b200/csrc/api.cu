@@ -40,7 +40,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
                      cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
-                     float* row_lse);
+                     float* row_lse, const int32_t* out_width);
 
 namespace {
 
@@ -98,7 +98,7 @@ extern "C" int beam_step(const sidbeam_trie* trie, int step, const void* logits,
                          void* stream) {
   return beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in, n_out,
                       V, out_scores, out_parent, out_code, out_node, workspace, workspace_bytes,
-                      stream, 0u);
+                      stream, 0u, nullptr);
 }
 
 extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
@@ -106,7 +106,7 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
                             const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
                             float* out_scores, int32_t* out_parent, int32_t* out_code,
                             int32_t* out_node, void* workspace, size_t workspace_bytes,
-                            void* stream, unsigned flags) {
+                            void* stream, unsigned flags, const int32_t* out_width) {
   if (flags & ~(static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS) | kValidateOnly))
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
   if (!logits || !parent_scores || !out_scores || !out_parent || !out_code || !out_node)
@@ -147,7 +147,7 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
                           workspace_bytes, static_cast<cudaStream_t>(stream), flags, 0.f, 0ull,
-                          nullptr);
+                          nullptr, out_width);
 }
 
 // Gumbel steps keep every row's lse after the beam_step workspace.
@@ -172,7 +172,7 @@ extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* 
   if (temperature == 0.f)  // the deterministic step
     return beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                         n_out, V, out_scores, out_parent, out_code, out_node, workspace,
-                        workspace_bytes, stream, 0u);
+                        workspace_bytes, stream, 0u, nullptr);
   const size_t need = beam_step_gumbel_workspace_size(R, B_in, n_out, V);
   if (need == 0 || workspace_bytes < need)
     return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step_gumbel: workspace of %zu bytes, need %zu",
@@ -180,14 +180,14 @@ extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* 
   // The shape checks of beam_step, then the Gumbel launch.
   const int rc = beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                               n_out, V, out_scores, out_parent, out_code, out_node, nullptr, 0,
-                              stream, kValidateOnly);
+                              stream, kValidateOnly, nullptr);
   if (rc != SIDBEAM_OK) return rc;
   float* row_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                             gumbel_lse_offset(R, B_in, n_out, V));
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
                           workspace_bytes, static_cast<cudaStream_t>(stream), 0u, temperature,
-                          seed, row_lse);
+                          seed, row_lse, nullptr);
 }
 
 extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,

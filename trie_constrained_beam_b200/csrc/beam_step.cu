@@ -105,6 +105,7 @@ struct StepArgs {
   uint32_t gseed0, gseed1;  // Philox key (seed lo, hi)
   int gstep;                // counter word 3
   float* row_lse;           // [R * B_in]: every live row's lse (the writer needs it)
+  const int32_t* out_width; // [R] beams kept per request (<= n), or null (n for all)
 };
 
 // ------------------------------------------------------------ Gumbel top-k
@@ -162,10 +163,11 @@ struct GumbelWriter {
   const float* parent_scores;
   const float* row_lse;
   int B_in;
+  const int32_t* width;
   __device__ __forceinline__ void operator()(int r, int i, uint64_t key, int32_t val,
                                              bool valid) const {
     const size_t o = static_cast<size_t>(r) * n + i;
-    if (valid) {
+    if (valid && (!width || i < width[r])) {
       const uint32_t idx = key_idx(key);
       const int32_t b = static_cast<int32_t>(idx / V), c = static_cast<int32_t>(idx % V);
       const int64_t row = static_cast<int64_t>(r) * B_in + b;
@@ -186,6 +188,8 @@ struct GumbelWriter {
   }
 };
 
+// Ranks at or past a request's width (out_width) are written as padding: the
+// top-w of a request are the first w ranks of its top-n.
 struct StepWriter {
   float* scores;
   int32_t* parent;
@@ -193,10 +197,11 @@ struct StepWriter {
   int32_t* node;
   int n;
   uint32_t V;
+  const int32_t* width;
   __device__ __forceinline__ void operator()(int r, int i, uint64_t key, int32_t val,
                                              bool valid) const {
     const size_t o = static_cast<size_t>(r) * n + i;
-    if (valid) {
+    if (valid && (!width || i < width[r])) {
       const uint32_t idx = key_idx(key);
       scores[o] = key_score(key);
       parent[o] = static_cast<int32_t>(idx / V);
@@ -1079,11 +1084,11 @@ __device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf w
   if constexpr (GUM) {
     const GumbelWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
                               static_cast<uint32_t>(a.V), a.logits, a.row_bytes, a.bf16,
-                              a.parent_scores, a.row_lse, a.B_in};
+                              a.parent_scores, a.row_lse, a.B_in, a.out_width};
     return segment_flush(team, wb, ctl, f, writer);
   } else {
     const StepWriter writer{a.out_scores, a.out_parent, a.out_code, a.out_node, a.n,
-                            static_cast<uint32_t>(a.V)};
+                            static_cast<uint32_t>(a.V), a.out_width};
     return segment_flush(team, wb, ctl, f, writer);
   }
 }
@@ -1588,7 +1593,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
                      cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
-                     float* row_lse) {
+                     float* row_lse, const int32_t* out_width) {
   StepArgs a{};
   a.logits = static_cast<const uint8_t*>(logits);
   a.bf16 = dtype == SIDBEAM_BF16;
@@ -1630,6 +1635,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   a.gseed1 = static_cast<uint32_t>(gumbel_seed >> 32);
   a.gstep = step;
   a.row_lse = row_lse;
+  a.out_width = out_width;
   a.tickets = reinterpret_cast<uint32_t*>(w + ws.tickets);
   a.request_thr = reinterpret_cast<unsigned long long*>(w + ws.request_thr);
   a.part_count = reinterpret_cast<uint32_t*>(w + ws.part_count);

@@ -82,7 +82,7 @@ def load():
     L.beam_step.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P]
     L.beam_step_noalloc.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P]
     L.beam_step_ex.argtypes = [P, I32, P, I32, I64, P, P, I32, I32, I32, I32, P, P, P, P, P, SZ, P,
-                               ctypes.c_uint]
+                               ctypes.c_uint, P]
     L.beam_step_skipped_rows.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
     L.beam_step_gumbel_workspace_size.argtypes = [I32, I32, I32, I32]
     L.beam_step_gumbel_workspace_size.restype = SZ
@@ -212,10 +212,11 @@ def beam_step_workspace_size(R: int, B_in: int, n_out: int, V: int) -> int:
 
 def beam_step(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V,
               out_scores, out_parent, out_code, out_node, workspace, stream=None, ld=None,
-              skip_rows=False):
+              skip_rows=False, out_width=None):
     """logits: torch [R*B_in, ld] float32/bfloat16 on the device (row stride = ld).
     skip_rows: do not read rows that cannot contribute (beam_step_ex with
-    SIDBEAM_STEP_SKIP_ROWS); the results are the same."""
+    SIDBEAM_STEP_SKIP_ROWS); the results are the same. out_width: optional
+    device int32 [R], beams kept per request (the rest of n_out is padding)."""
     if ld is None:
         ld = logits.stride(0)
     args = (None if trie is None else trie.handle, step, _ptr(logits), _dtype_code(logits), ld,
@@ -223,8 +224,9 @@ def beam_step(trie, step, logits, parent_scores, parent_nodes, R, B_in, n_out, V
             _ptr(out_parent), _ptr(out_code), _ptr(out_node), _ptr(workspace),
             0 if workspace is None else workspace.numel() * workspace.element_size(),
             _stream(stream))
-    if skip_rows:
-        rc = load().beam_step_ex(*args, STEP_SKIP_ROWS)
+    if skip_rows or out_width is not None:
+        rc = load().beam_step_ex(*args, STEP_SKIP_ROWS if skip_rows else 0,
+                                 None if out_width is None else _ptr(out_width))
     else:
         rc = load().beam_step(*args)
     _check(rc)

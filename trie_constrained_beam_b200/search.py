@@ -14,7 +14,12 @@ from . import native
 
 class BeamSearch:
     def __init__(self, trie, R: int, n: int, V, depth: int = None, device="cuda",
-                 skip_rows: bool = False, temperature: float = 0.0, seed: int = 0):
+                 skip_rows: bool = False, temperature: float = 0.0, seed: int = 0,
+                 widths=None):
+        """widths: optional per-request beam widths (each <= n); request r keeps
+        its widths[r] best beams at every step (the rest of its n slots are
+        padding), so one launch per step and one captured graph serve requests
+        of different widths."""
         self.trie = trie
         self.skip_rows = skip_rows  # beam_step_ex row skipping (same results)
         # temperature > 0: Gumbel top-k draws (beam_step_gumbel), Philox key `seed`
@@ -35,6 +40,14 @@ class BeamSearch:
                     else native.beam_step_workspace_size)
             ws = max(ws, size(R, 1 if t == 0 else n, n, self.V[t]))
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=dev)
+        self.widths = None
+        if widths is not None:
+            w = [int(x) for x in widths]
+            if len(w) != R or min(w) < 0 or max(w) > n:
+                raise ValueError("widths: one value in [0, n] per request")
+            if self.temperature > 0:
+                raise ValueError("widths with temperature > 0 is not supported")
+            self.widths = torch.tensor(w, dtype=torch.int32, device=dev)
         self.sids = torch.empty((R, n, self.depth), dtype=torch.int32, device=dev)
         self.leaf = torch.empty((R, n), dtype=torch.int32, device=dev)
 
@@ -57,7 +70,8 @@ class BeamSearch:
             return
         native.beam_step(self.trie, t, logits, ps, pn, self.R, B_in, self.n, self.V[t],
                          self.scores[t], self.bp_parent[t], self.bp_code[t], self.nodes[t],
-                         self.workspace, stream=stream, skip_rows=self.skip_rows)
+                         self.workspace, stream=stream, skip_rows=self.skip_rows,
+                         out_width=self.widths)
 
     def skipped_rows(self, stream=None) -> int:
         """Rows left unread by row skipping since the last call."""
