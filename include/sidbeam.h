@@ -164,9 +164,9 @@ int beam_step(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dt
               void* stream);
 
 /* beam_step_ex -- beam_step with options (flags: OR of SIDBEAM_STEP_*).
- *  SIDBEAM_STEP_SKIP_ROWS: row skipping (the first of the "next" items, not a
- *  step the pages describe; it leaves every result unchanged). Every child's
- *  score s + (z - lse) is at most its parent's score s (z <= lse), so a row
+ *  SIDBEAM_STEP_SKIP_ROWS: row skipping (not a step the pages describe; it
+ *  leaves every result unchanged). Every child's score s + (z - lse) is at
+ *  most its parent's score s (z <= lse), so a row
  *  whose parent score cannot reach a valid lower bound on the request's n-th
  *  best key that the step already holds can contribute nothing: its logits
  *  are not read. Applies when the request's rows are spread over CTAs that
@@ -178,8 +178,9 @@ int beam_step(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dt
  *  (score -inf, indices -1), so they are dead rows of the next step and are
  *  never read. The kept beams are exactly the first out_width[r] ranks of the
  *  request's top n_out, the same as a step with n_out = out_width[r]: per-request
- *  beam widths in one launch (and so in one captured graph of the whole search;
- *  the third of the "next" items). Values outside [0, n_out] are undefined.
+ *  beam widths in one launch, and so in one captured graph of the whole search
+ *  (flashrec 0.1.0, Features > Decoding, "Scheduling": rows of several requests
+ *  share a step). Values outside [0, n_out] are undefined.
  *  Other arguments, results and errors: those of beam_step; unknown flag bits
  *  give INVALID_ARG. beam_step(...) is beam_step_ex(..., 0, NULL). */
 #define SIDBEAM_STEP_SKIP_ROWS 1u
@@ -190,9 +191,9 @@ int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits, sidbeam
                  void* stream, unsigned flags, const int32_t* out_width);
 
 /* beam_step_gumbel -- beam_step at temperature > 0: Gumbel top-k without
- * replacement (flashrec 0.1.0, Features > Serving, "API"; the second of the
- * "next" items). Candidate c of parent slot b in request r, with the usual
- * score x = s_b + (z_c - lse_b), is ranked by the key x + T*G, G = -log(-log U)
+ * replacement (flashrec 0.1.0, Features > Serving, "API"). Candidate c of
+ * parent slot b in request r, with the usual score x = s_b + (z_c - lse_b), is
+ * ranked by the key x + T*G, G = -log(-log U)
  * a standard Gumbel variate: U = (v + 1/2) * 2^-23 with v the top 23 bits of
  * the first output word of Philox4x32-10 (Salmon et al., SC'11) on the counter
  * (r, b, c, step) with key (seed low 32 bits, seed high 32 bits). The n largest
