@@ -94,3 +94,21 @@ def test_workspace_size_shapes(lib):
     a = native.beam_step_workspace_size(16, 512, 512, 4096)
     b = native.beam_step_workspace_size(16, 512, 256, 4096)
     assert a > b > 0 and a % 256 == 0
+
+
+def test_step_options_argument_checks(lib):
+    """beam_step_ex, beam_step_gumbel and catalog_score_topk_sim reject bad
+    arguments on the host (no device call is made on these paths)."""
+    P = ctypes.c_void_p
+    base = (None, 0, P(0x1000), 0, 64, P(0x2000), P(0x3000), 1, 1, 4, 64, P(0x4000), P(0x5000),
+            P(0x6000), P(0x7000), P(0x8000), 1 << 20, None)
+    assert lib.beam_step_ex(*base, 0x4, None) == -1          # unknown flag bit
+    assert lib.beam_step_ex(*base[:9], 0, *base[10:], 0, None) == -1   # n_out = 0
+    g = (None, 0, P(0x1000), 0, 64, P(0x2000), P(0x3000), 1, 1, 4, 64)
+    outs = (P(0x4000), P(0x5000), P(0x6000), P(0x7000), P(0x8000), 1 << 20, None)
+    for T in (-1.0, float("nan"), float("inf")):
+        assert lib.beam_step_gumbel(*g, ctypes.c_float(T), ctypes.c_uint64(1), *outs) == -1
+    assert lib.beam_step_gumbel(*g, ctypes.c_float(1.0), ctypes.c_uint64(1),
+                                *outs[:5], 16, None) == -4            # workspace too small
+    assert lib.catalog_score_topk_sim(None, P(0x1000), P(0x2000), P(0x3000), 8, 1, 1,
+                                      P(0x4000), P(0x5000), P(0x6000), 1 << 20, None) == -1
