@@ -17,8 +17,10 @@ scores and the step is the deterministic one.
 
 The Gumbel variate: Philox4x32 with ten rounds (Salmon, Moraes, Dror, Shaw,
 SC'11, "Parallel random numbers: as easy as 1, 2, 3") on the counter
-(r, b, c, step) with the 64-bit seed as key; its first output word u gives
-U = (u + 1/2) / 2^32 in (0, 1) and G = -log(-log U).
+(r, b, c, step) with the 64-bit seed as key; the top 23 bits of its first
+output word, v = u >> 9, give U = (v + 1/2) / 2^23 in (0, 1) (exact in fp32, so a
+device in single precision sees the same U) and G = -log(-log U), which lies in
+[-2.82, 16.64].
 
 TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 """
@@ -55,7 +57,7 @@ def philox4x32_10(c0, c1, c2, c3, k0: int, k1: int):
 def gumbel(seed: int, r, b, code, step: int) -> np.ndarray:
     """Standard Gumbel variates for candidates (r, b, code) of `step` (float64)."""
     u = philox4x32_10(r, b, code, step, seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)[0]
-    U = (u.astype(np.float64) + 0.5) / 4294967296.0
+    U = ((u >> np.uint32(9)).astype(np.float64) + 0.5) / 8388608.0
     return -np.log(-np.log(U))
 
 
