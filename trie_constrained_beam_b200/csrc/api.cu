@@ -101,14 +101,13 @@ extern "C" int beam_step(const sidbeam_trie* trie, int step, const void* logits,
                       stream, 0u, nullptr);
 }
 
-extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
-                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
-                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
-                            float* out_scores, int32_t* out_parent, int32_t* out_code,
-                            int32_t* out_node, void* workspace, size_t workspace_bytes,
-                            void* stream, unsigned flags, const int32_t* out_width) {
-  if (flags & ~(static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS) | kValidateOnly))
-    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
+// The host checks every step entry point shares (shapes, pointers, alignment).
+static int check_step_args(const sidbeam_trie* trie, int step, const void* logits,
+                           sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                           const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                           const float* out_scores, const int32_t* out_parent,
+                           const int32_t* out_code, const int32_t* out_node,
+                           const void* workspace) {
   if (!logits || !parent_scores || !out_scores || !out_parent || !out_code || !out_node)
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: NULL pointer argument");
   if (trie && !parent_nodes)
@@ -143,7 +142,21 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
   }
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step: workspace must be 256-byte aligned");
-  if (flags & kValidateOnly) return SIDBEAM_OK;
+  return SIDBEAM_OK;
+}
+
+extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
+                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                            float* out_scores, int32_t* out_parent, int32_t* out_code,
+                            int32_t* out_node, void* workspace, size_t workspace_bytes,
+                            void* stream, unsigned flags, const int32_t* out_width) {
+  if (flags & ~static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS))
+    return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
+  const int rc = check_step_args(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R,
+                                 B_in, n_out, V, out_scores, out_parent, out_code, out_node,
+                                 workspace);
+  if (rc != SIDBEAM_OK) return rc;
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
                           workspace_bytes, static_cast<cudaStream_t>(stream), flags, 0.f, 0ull,
@@ -178,9 +191,9 @@ extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* 
     return set_error(SIDBEAM_ERR_WORKSPACE, "beam_step_gumbel: workspace of %zu bytes, need %zu",
                      workspace_bytes, need);
   // The shape checks of beam_step, then the Gumbel launch.
-  const int rc = beam_step_ex(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
-                              n_out, V, out_scores, out_parent, out_code, out_node, nullptr, 0,
-                              stream, kValidateOnly, nullptr);
+  const int rc = check_step_args(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R,
+                                 B_in, n_out, V, out_scores, out_parent, out_code, out_node,
+                                 workspace);
   if (rc != SIDBEAM_OK) return rc;
   float* row_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                             gumbel_lse_offset(R, B_in, n_out, V));

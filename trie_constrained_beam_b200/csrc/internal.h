@@ -54,7 +54,5 @@ constexpr uint32_t kStatusTimeout = 2u;
 constexpr size_t kSkippedRowsOffset = 8;
 // ... and of max_j ||e_j|| for catalog_score_topk_sim (written each call).
 constexpr size_t kEmbNormOffset = 16;
-// beam_step_ex flag used inside the library: check the arguments, launch nothing.
-constexpr unsigned kValidateOnly = 0x80000000u;
 
 }  // namespace sidbeam
