@@ -161,18 +161,19 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
         if (SIM) {  // <u_r, e_j>: 16-byte loads of the leaf's bf16 row, four partial sums
           const uint4* er = reinterpret_cast<const uint4*>(a.emb + j * a.d);
           float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+          const float4* u4 = reinterpret_cast<const float4*>(user);  // 16-byte aligned region
 #pragma unroll 2
           for (int k8 = 0; k8 < (a.d >> 3); ++k8) {
             const uint4 q = __ldg(er + k8);
-            const float* uk = user + k8 * 8;
-            d0 = fmaf(__uint_as_float(q.x << 16), uk[0], d0);
-            d1 = fmaf(__uint_as_float(q.x & 0xFFFF0000u), uk[1], d1);
-            d2 = fmaf(__uint_as_float(q.y << 16), uk[2], d2);
-            d3 = fmaf(__uint_as_float(q.y & 0xFFFF0000u), uk[3], d3);
-            d0 = fmaf(__uint_as_float(q.z << 16), uk[4], d0);
-            d1 = fmaf(__uint_as_float(q.z & 0xFFFF0000u), uk[5], d1);
-            d2 = fmaf(__uint_as_float(q.w << 16), uk[6], d2);
-            d3 = fmaf(__uint_as_float(q.w & 0xFFFF0000u), uk[7], d3);
+            const float4 ua = u4[2 * k8], ub = u4[2 * k8 + 1];  // broadcast loads
+            d0 = fmaf(__uint_as_float(q.x << 16), ua.x, d0);
+            d1 = fmaf(__uint_as_float(q.x & 0xFFFF0000u), ua.y, d1);
+            d2 = fmaf(__uint_as_float(q.y << 16), ua.z, d2);
+            d3 = fmaf(__uint_as_float(q.y & 0xFFFF0000u), ua.w, d3);
+            d0 = fmaf(__uint_as_float(q.z << 16), ub.x, d0);
+            d1 = fmaf(__uint_as_float(q.z & 0xFFFF0000u), ub.y, d1);
+            d2 = fmaf(__uint_as_float(q.w << 16), ub.z, d2);
+            d3 = fmaf(__uint_as_float(q.w & 0xFFFF0000u), ub.w, d3);
           }
           score += (d0 + d1) + (d2 + d3);
         }
