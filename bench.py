@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -183,8 +184,10 @@ def run_ours(args, world, rank, local):
 
     K = args.steps
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, "/tmp/_clk.csv")
+    # Raw nvidia-smi samples go to --clocks-dir (kept) or a temporary file; the
+    # JSON line carries their summary either way.
+    clk_dir = args.clocks_dir or tempfile.gettempdir()
+    clocks = ClockSampler(local, os.path.join(clk_dir, f"clocks_rank{rank}.csv"))
     time.sleep(0.3)
     if world > 1:
         torch.distributed.barrier()
@@ -625,6 +628,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused lm_head (tcgen05) lines")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="directory for the raw clock samples (default: a temporary directory)")
     ap.add_argument("--no-widths", action="store_true",
                     help="skip the per-request widths line")
     ap.add_argument("--no-gumbel", action="store_true",
