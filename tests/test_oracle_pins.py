@@ -342,6 +342,24 @@ def test_catalog_scorer_zero_embeddings_is_token_only():
     assert np.array_equal(a["leaf"], b["leaf"]) and np.array_equal(a["score"], b["score"])
 
 
+def test_catalog_scorer_zero_table_ranks_by_similarity():
+    """With every token log-probability 0 the ranking is the similarity's alone:
+    the SIDs sorted by the dot product, written out per SID."""
+    Vs = [8, 8]
+    cat = host.draw_catalog(12, 40, Vs)
+    trie = oracle.OracleTrie(cat, Vs)
+    d = 16
+    user = host.user_vectors(12, 2, d, 1.0)
+    emb = host.sid_embeddings(12, trie.leaves.shape[0], d, 0.3)
+    ef = host.bf16_bits_to_f32(emb)
+    res = oracle.catalog_score_topk(trie, np.zeros((2, 2, 8)), 40, user, emb)
+    for r in range(2):
+        dots = [(sum(float(user[r, k]) * float(ef[j, k]) for k in range(d)), j)
+                for j in range(trie.leaves.shape[0])]
+        dots.sort(key=lambda x: (-x[0], x[1]))
+        assert res["leaf"][r].tolist() == [j for _, j in dots]
+
+
 # ------------------------------------------------------------------ Gumbel top-k
 def test_oracle_philox_known_answers():
     """The oracle's own Philox4x32-10 against the published known-answer vectors."""
