@@ -52,6 +52,18 @@ def _dist():
     return world, rank, local
 
 
+def _max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's x: a collective, so every rank calls it at
+    the same point (one process: x itself)."""
+    import torch
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _workload_config(w, extra=None):
     cfg = {
         "workload": w.name,
@@ -200,11 +212,7 @@ def run_ours(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    elapsed_ms = start.elapsed_time(stop)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = _max_over_ranks(start.elapsed_time(stop), dev)
     assert torch.equal(search.sids, ref_sids)
     assert tcb.sidbeam_get_device_status(search.workspace) == 0
 
@@ -260,11 +268,7 @@ def run_ours(args, world, rank, local):
             e2e_search()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = _max_over_ranks(e0.elapsed_time(e1), dev)
         assert torch.equal(out_sids, ref_sids.cpu())
         h2d = sum(x.numel() * x.element_size() for x in pinned)
         d2h = out_sids.numel() * 4 + out_leaf.numel() * 4 + out_score.numel() * 4
