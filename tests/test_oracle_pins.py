@@ -360,6 +360,47 @@ def test_catalog_scorer_zero_table_ranks_by_similarity():
         assert res["leaf"][r].tolist() == [j for _, j in dots]
 
 
+def _random_step_case(seed, V=24, n_cat=400, R=3, B_in=20):
+    rng = np.random.default_rng(seed)
+    cat = host.draw_catalog(seed, n_cat, [V, V])
+    trie = oracle.OracleTrie(cat, [V, V])
+    z = rng.normal(0, 2, size=(R * B_in, V))
+    ps = np.concatenate([np.sort(rng.uniform(-9, -1, size=B_in))[::-1] for _ in range(R)])
+    pn = rng.integers(0, trie.n_nodes(1), size=R * B_in)
+    return trie, z, ps, pn, R, B_in, V
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_rows_below_the_nth_best_never_contribute(seed):
+    """The fact row skipping rests on: a child's score never exceeds its
+    parent's (log p <= 0), so dropping every row whose parent score is below
+    the request's n-th best child leaves the step's result unchanged."""
+    trie, z, ps, pn, R, B_in, V = _random_step_case(200 + seed)
+    n = 8
+    full = oracle.beam_step(trie, 1, z, ps, pn, R, B_in, n, V)
+    cut = ps.copy()
+    for r in range(R):
+        kth = full["score"][r, n - 1]
+        rows = slice(r * B_in, (r + 1) * B_in)
+        cut[rows] = np.where(ps[rows] < kth, -np.inf, ps[rows])
+    assert np.isneginf(cut).any()          # the case does drop rows
+    pruned = oracle.beam_step(trie, 1, z, cut, pn, R, B_in, n, V)
+    for k in ("score", "parent", "code", "node"):
+        assert np.array_equal(full[k], pruned[k])
+
+
+def test_top_w_is_the_first_w_ranks_of_top_n():
+    """The fact per-request widths rest on: the best w candidates of a request
+    are the first w ranks of its best n (n >= w), ties included."""
+    trie, z, ps, pn, R, B_in, V = _random_step_case(300)
+    z = np.round(z * 2) / 2                 # coarse grid: many exact ties
+    wide = oracle.beam_step(trie, 1, z, ps, pn, R, B_in, 40, V)
+    for w in (1, 7, 23, 40):
+        narrow = oracle.beam_step(trie, 1, z, ps, pn, R, B_in, w, V)
+        for k in ("score", "parent", "code", "node"):
+            assert np.array_equal(wide[k][:, :w], narrow[k])
+
+
 # ------------------------------------------------------------------ Gumbel top-k
 def test_oracle_philox_known_answers():
     """The oracle's own Philox4x32-10 against the published known-answer vectors."""
