@@ -112,3 +112,20 @@ def test_step_options_argument_checks(lib):
                                 *outs[:5], 16, None) == -4            # workspace too small
     assert lib.catalog_score_topk_sim(None, P(0x1000), P(0x2000), P(0x3000), 8, 1, 1,
                                       P(0x4000), P(0x5000), P(0x6000), 1 << 20, None) == -1
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/sidbeam.h compiles on its own as C99 (pedantic): no C++ or CUDA
+    types leak into the boundary."""
+    import shutil
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "sidbeam.h"\n'
+                   "int main(void) { sidbeam_trie* t = 0; (void)t;\n"
+                   "  return (int)beam_step_workspace_size(1, 1, 1, 1) * 0; }\n")
+    import subprocess
+    out = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                          "-I", os.path.join(ROOT, "include"), "-c", str(src), "-o",
+                          str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
