@@ -1,0 +1,41 @@
+// Test harness (host only): exposes the row partition of the launch geometry
+// header to the CPU tests. Built by tests/test_partition_host.py with g++.
+#include <stdint.h>
+
+#include "launch.h"
+
+// For every CTA c, writes each row of its sequence (rows(c, 0, 1)) into rows[]
+// (CTA-major, `cap` slots per CTA, count in counts[c]); for every warp w < W,
+// the warp's share (rows(c, w, W)) is checked to be the CTA entries w, w + W, ...
+// Returns the grid size, or -1 when a warp share disagrees or a CTA has more
+// than `cap` rows. maxG and the per-request contributor counts are returned too.
+extern "C" int partition_probe(int R, int64_t B_in, int ctas, int W, int cap, int64_t* rows,
+                               int* counts, int* maxG, int* first_cta, int* last_cta,
+                               int* contributors) {
+  const sidbeam::Partition p = sidbeam::make_partition(R, B_in, ctas);
+  *maxG = p.maxG;
+  for (int r = 0; r < R; ++r) {
+    first_cta[r] = p.first_cta(r);
+    last_cta[r] = p.last_cta(r);
+    contributors[r] = p.contributors(r);
+  }
+  for (int c = 0; c < p.grid; ++c) {
+    int64_t first, stride;
+    int count;
+    p.rows(c, 0, 1, first, stride, count);
+    if (count > cap) return -1;
+    counts[c] = count;
+    for (int i = 0; i < count; ++i) rows[static_cast<int64_t>(c) * cap + i] = first + stride * i;
+    for (int w = 0; w < W; ++w) {
+      int64_t f2, s2;
+      int n2;
+      p.rows(c, w, W, f2, s2, n2);
+      int expect = 0;
+      for (int i = w; i < count; i += W) ++expect;
+      if (n2 != expect) return -1;
+      for (int k = 0; k < n2; ++k)
+        if (f2 + s2 * k != first + stride * (w + static_cast<int64_t>(W) * k)) return -1;
+    }
+  }
+  return p.grid;
+}

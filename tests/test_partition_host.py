@@ -1,0 +1,71 @@
+"""Host-side row partition over CTAs (the launch geometry every kernel uses),
+checked on the CPU: every row goes to exactly one CTA, a CTA of a request
+group holds only that request's rows, contiguous chunks stay contiguous, the
+warps' shares are the CTA's entries w, w + W, ..., and the contributor counts
+and first/last CTAs of each request agree with the rows and stay within maxG."""
+import ctypes
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def probe(tmp_path_factory):
+    cuda_inc = "/usr/local/cuda/include"
+    if shutil.which("g++") is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("needs g++ and the CUDA headers")
+    out = tmp_path_factory.mktemp("probe") / "partition_probe.so"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-shared", "-fPIC", "-I", cuda_inc,
+                    "-I", os.path.join(ROOT, "trie_constrained_beam_b200", "csrc"),
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "host", "partition_probe.cpp"), "-o", str(out)],
+                   check=True)
+    lib = ctypes.CDLL(str(out))
+    P = ctypes.c_void_p
+    lib.partition_probe.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, P, P, P, P, P, P]
+    lib.partition_probe.restype = ctypes.c_int
+    return lib
+
+
+@pytest.mark.parametrize("R,B_in,ctas", [(16, 512, 148), (16, 1, 148), (64, 128, 148),
+                                         (1, 2000, 148), (160, 40, 148), (1000, 3, 148),
+                                         (3, 7, 148), (32, 32, 592), (7, 100000, 148)])
+def test_partition_covers_every_row_once(probe, R, B_in, ctas):
+    W = 12
+    cap = max(1, -(-R * B_in // min(ctas, R * B_in))) + B_in + 1
+    grid_max = ctas
+    rows = np.full(grid_max * cap, -1, dtype=np.int64)
+    counts = np.zeros(grid_max, dtype=np.int32)
+    maxG = np.zeros(1, dtype=np.int32)
+    first = np.zeros(R, dtype=np.int32)
+    last = np.zeros(R, dtype=np.int32)
+    contrib = np.zeros(R, dtype=np.int32)
+    grid = probe.partition_probe(R, B_in, ctas, W, cap, rows.ctypes.data, counts.ctypes.data,
+                                 maxG.ctypes.data, first.ctypes.data, last.ctypes.data,
+                                 contrib.ctypes.data)
+    assert 0 < grid <= ctas
+    seen = np.zeros(R * B_in, dtype=np.int32)
+    ctas_of = [set() for _ in range(R)]
+    grouped = R <= ctas
+    for c in range(grid):
+        got = rows[c * cap:c * cap + counts[c]]
+        assert np.all((got >= 0) & (got < R * B_in))
+        np.add.at(seen, got, 1)
+        reqs = set((got // B_in).tolist())
+        for r in reqs:
+            ctas_of[r].add(c)
+        if grouped:
+            assert len(reqs) <= 1                         # one request per CTA
+        elif counts[c]:
+            assert np.array_equal(got, np.arange(got[0], got[0] + counts[c]))  # contiguous
+    assert np.all(seen == 1)                              # every row exactly once
+    for r in range(R):
+        # the CTAs holding rows of r are exactly first..last, at most maxG of them
+        assert ctas_of[r] == set(range(first[r], last[r] + 1))
+        assert contrib[r] == last[r] - first[r] + 1 <= maxG[0]
