@@ -39,3 +39,12 @@ extern "C" int partition_probe(int R, int64_t B_in, int ctas, int W, int cap, in
   }
   return p.grid;
 }
+
+// The workspace carve-up: offsets of status, tickets, request_thr, ghist,
+// part_count, part_keys, part_vals and the total, in that order.
+extern "C" void workspace_probe(int R, int maxG, int n, int64_t* out) {
+  const sidbeam::WorkspaceLayout w = sidbeam::workspace_layout(R, maxG, n);
+  const size_t v[8] = {w.status, w.tickets, w.request_thr, w.ghist, w.part_count,
+                       w.part_keys, w.part_vals, w.total};
+  for (int i = 0; i < 8; ++i) out[i] = static_cast<int64_t>(v[i]);
+}

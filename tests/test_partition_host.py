@@ -69,3 +69,22 @@ def test_partition_covers_every_row_once(probe, R, B_in, ctas):
         # the CTAs holding rows of r are exactly first..last, at most maxG of them
         assert ctas_of[r] == set(range(first[r], last[r] + 1))
         assert contrib[r] == last[r] - first[r] + 1 <= maxG[0]
+
+
+@pytest.mark.parametrize("R,maxG,n", [(16, 9, 512), (1, 148, 4096), (1000, 2, 3), (64, 2, 128)])
+def test_workspace_layout_parts_fit(probe, R, maxG, n):
+    """Every part starts 256-byte aligned, after the end of the one before, and
+    the total covers the last: [status 4 B | tickets R x 4 | request bounds R x 8
+    | histograms R x 1024 x 4 | part counts R x maxG x 4 | part keys R x maxG x 2n
+    x 8 | part values R x maxG x 2n x 4]."""
+    probe.workspace_probe.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    probe.workspace_probe.restype = None
+    out = np.zeros(8, dtype=np.int64)
+    probe.workspace_probe(R, maxG, n, out.ctypes.data)
+    sizes = [4, R * 4, R * 8, R * 1024 * 4, R * maxG * 4, R * maxG * 2 * n * 8,
+             R * maxG * 2 * n * 4]
+    assert out[0] == 0
+    for i in range(7):
+        assert out[i] % 256 == 0
+        end = out[i] + sizes[i]
+        assert (out[i + 1] if i < 6 else out[7]) >= end
