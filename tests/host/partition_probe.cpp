@@ -48,3 +48,21 @@ extern "C" void workspace_probe(int R, int maxG, int n, int64_t* out) {
                        w.part_keys, w.part_vals, w.total};
   for (int i = 0; i < 8; ++i) out[i] = static_cast<int64_t>(v[i]);
 }
+
+#include "step_plan.h"
+
+// The beam_step shared-memory plan for one shape: returns whether one fits and
+// writes W, S, Cw, stage_bytes, logits_copy_bytes, the ten region offsets
+// (ctl, bars, meta, chist, whist, wprefix, wmask, stage, wkeys, wvals) and
+// smem_bytes, in that order (17 ints).
+extern "C" int plan_probe(int V, int esize, int extra, int prefix_words, int n, int reg,
+                          int ctl_bytes, int* out) {
+  sidbeam::StepConfig c{};
+  if (!sidbeam::choose_step_config(V, esize, extra, prefix_words, n, reg != 0, ctl_bytes, &c))
+    return 0;
+  const int v[17] = {c.W, c.S, c.Cw, c.stage_bytes, c.logits_copy_bytes, c.off_ctl, c.off_bars,
+                     c.off_meta, c.off_chist, c.off_whist, c.off_wprefix, c.off_wmask,
+                     c.off_stage, c.off_wkeys, c.off_wvals, c.smem_bytes, c.reg};
+  for (int i = 0; i < 17; ++i) out[i] = v[i];
+  return 1;
+}

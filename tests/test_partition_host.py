@@ -88,3 +88,40 @@ def test_workspace_layout_parts_fit(probe, R, maxG, n):
         assert out[i] % 256 == 0
         end = out[i] + sizes[i]
         assert (out[i + 1] if i < 6 else out[7]) >= end
+
+
+# (V, bytes per logit, trie bytes staged per row, mask words per warp, n): the
+# step shapes of the five workloads, plus edge shapes.
+_SHAPES = [(32, 4, 512, 4, 8), (32, 4, 512, 4, 2000), (256, 4, 32, 8, 32), (256, 4, 512, 8, 32),
+           (8192, 2, 512, 256, 128), (4096, 2, 512, 128, 512), (4096, 2, 512, 128, 4096),
+           (8192, 4, 512, 256, 64), (1, 4, 0, 0, 1), (16384, 4, 512, 512, 16)]
+
+
+@pytest.mark.parametrize("shape", _SHAPES)
+@pytest.mark.parametrize("ctl_bytes", [7424, 12288])
+def test_step_plan_regions_aligned_and_disjoint(probe, shape, ctl_bytes):
+    """Every region of the plan is aligned for how it is accessed (bulk-copy
+    stages and their sizes on 128 bytes, the parent table and mask copies read
+    as 16-byte vectors, 64-bit keys), the regions follow one another without
+    overlap, and the whole plan fits the 227 KiB budget."""
+    V, esize, extra, pw, n = shape
+    probe.plan_probe.argtypes = [ctypes.c_int] * 7 + [ctypes.c_void_p]
+    probe.plan_probe.restype = ctypes.c_int
+    for reg in ((0, 1) if V * esize <= 8192 else (0,)):
+        out = np.zeros(17, dtype=np.int32)
+        if not probe.plan_probe(V, esize, extra, pw, n, reg, ctl_bytes, out.ctypes.data):
+            assert n > 2000 or reg  # only a huge n (or the register plan) may not fit
+            continue
+        W, S, Cw, sb, lcb, ctl, bars, meta, chist, whist, wpre, wmask, stage, wkeys, wvals, smem, rg = (
+            int(x) for x in out)
+        assert 1 <= W <= 12 and 1 <= S <= 8 and Cw >= n + 32 and rg == reg
+        assert lcb >= V * esize and lcb % 16 == 0 and sb >= lcb + extra and sb % 128 == 0
+        for off, a in ((ctl, 128), (bars, 128), (meta, 16), (chist, 16), (whist, 16),
+                       (wpre, 16), (wmask, 16), (stage, 128), (wkeys, 128), (wvals, 16)):
+            assert off % a == 0
+        ends = [(ctl, ctl_bytes), (bars, W * 8 * 8), (meta, 256 * 16), (chist, 1024),
+                (whist, max(W * 1024, 2 * 1024 * 4)), (wpre, W * pw * 4), (wmask, W * pw * 4),
+                (stage, W * S * sb), (wkeys, W * Cw * 8), (wvals, W * Cw * 4)]
+        for (o1, n1), (o2, _) in zip(ends, ends[1:]):
+            assert o1 + n1 <= o2
+        assert wvals + W * Cw * 4 <= smem <= 232448

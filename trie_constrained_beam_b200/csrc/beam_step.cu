@@ -36,6 +36,7 @@
 #include "device_utils.cuh"
 #include "internal.h"
 #include "launch.h"
+#include "step_plan.h"
 #include "topn.cuh"
 
 namespace sidbeam {
@@ -960,10 +961,6 @@ __device__ void smem_walk(const StepArgs& a, const uint8_t* zrow, const RowCtx& 
   }
 }
 
-// Rows of a CTA whose parent data fits the shared table: up to this many, the
-// warps take rows from a shared counter instead of a fixed share each.
-constexpr int kMetaRows = 256;
-
 // Moves this CTA's histogram counts into request r's global histogram and
 // raises the shared bounds from the global one, which holds every CTA's
 // pushed counts (warp-collective; one warp of the CTA at a time, the others
@@ -1502,73 +1499,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
 // ------------------------------------------------------------------ host side
 
 static int round_up(int x, int m) { return (x + m - 1) / m * m; }
-
-// Shared-memory plan: [control | barriers | radix scratch | warp histograms
-// (>= 2 x 1024 words: the rank merge's scratch) | dense prefix counts | mask
-// copies | W x S stages | W top-n buffers]. The first warp count (from 8 down)
-// that fits with at least two stages per warp wins; one stage per warp is the
-// last resort. Small rows get more stages (up to kMaxStages).
-bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int n, bool reg,
-                        StepConfig* cfg) {
-  StepConfig c{};
-  c.logits_copy_bytes = round_up(V * esize, 16);
-  c.extra_bytes = extra_bytes;
-  c.stage_bytes = round_up(c.logits_copy_bytes + extra_bytes, 128);
-  c.prefix_words = prefix_words;
-  c.reg = reg ? 1 : 0;
-  int npow2 = 1;
-  while (npow2 < n) npow2 <<= 1;
-  const int ctl_bytes = round_up(static_cast<int>(sizeof(dev::SelCtl)), 128);
-  // Register rows: 12 warps with one stage each (more warps hide more
-  // latency; the stage is refilled as soon as the row is in registers).
-  // Rows worked on in place: at least two stages per warp.
-  struct Plan { int W, min_s; };
-  static const Plan kRegPlans[] = {{12, 1}, {8, 2}, {8, 1}, {6, 1}, {4, 1}, {2, 1}, {1, 1}};
-  static const Plan kSmemPlans[] = {{8, 2}, {6, 2}, {4, 2}, {8, 1}, {6, 1}, {4, 1}, {2, 1}, {1, 1}};
-  const Plan* plans = reg ? kRegPlans : kSmemPlans;
-  const int nplans = reg ? 7 : 8;
-  for (int pi = 0; pi < nplans; ++pi) {
-    {
-      const int W = plans[pi].W, min_s = plans[pi].min_s;
-      if (W > (reg ? kMaxStepWarpsReg : kMaxStepWarps)) continue;
-      const int cw = std::max(round_up(n, 32) + 32, round_up((npow2 + W - 1) / W, 32));
-      int o = 0;
-      c.off_ctl = o;
-      o += ctl_bytes;
-      c.off_bars = o;
-      o += round_up(W * kMaxStages * 8, 128);
-      c.off_meta = o;
-      o += kMetaRows * 16;
-      c.off_chist = o;
-      o += 1024;
-      c.off_whist = o;
-      o += std::max(W * 1024, 2 * dev::kHistBins * 4);
-      c.off_wprefix = o;
-      o += W * c.prefix_words * 4;
-      c.off_wmask = o;
-      o += W * c.prefix_words * 4;
-      o = round_up(o, 128);
-      const int warp_bytes = W * cw * 12 + 256;
-      const int avail = kSmemBudget - o - warp_bytes;
-      const int S = std::min(kMaxStages, avail / (W * c.stage_bytes));
-      if (S < min_s) continue;
-      c.W = W;
-      c.S = S;
-      c.Cw = cw;
-      c.off_stage = o;
-      o += W * S * c.stage_bytes;
-      c.off_wkeys = round_up(o, 128);
-      o = c.off_wkeys + W * cw * 8;
-      c.off_wvals = round_up(o, 16);
-      o = c.off_wvals + W * cw * 4;
-      c.smem_bytes = round_up(o, 128);
-      if (c.smem_bytes > kSmemBudget) continue;
-      *cfg = c;
-      return true;
-    }
-  }
-  return false;
-}
+static_assert(dev::kHistBins == kPlanHistBins, "the plan sizes the rank-merge scratch");
 
 // Raise the kernel's dynamic shared-memory limit to the full budget once per
 // device (kept out of the per-call path, and out of any stream capture that
@@ -1651,8 +1582,10 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                                  : (a.layout == SIDBEAM_LAYOUT_CSR ? ((V + 31) / 32 + 3) / 4 * 4 : 0);
   // (Gumbel steps walk every row in shared memory.)
   const bool reg = !gum && static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
-  if (!choose_step_config(V, esize, extra, prefix_words, n_out, reg, &a.cfg) &&
-      !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, &a.cfg)))
+  const int ctl_bytes = round_up(static_cast<int>(sizeof(dev::SelCtl)), 128);
+  if (!choose_step_config(V, esize, extra, prefix_words, n_out, reg, ctl_bytes, &a.cfg) &&
+      !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, ctl_bytes,
+                                  &a.cfg)))
     return set_error(SIDBEAM_ERR_INVALID_ARG,
                      "beam_step: V=%d with n_out=%d does not fit in shared memory", V, n_out);
   if (a.cfg.W > (a.cfg.reg ? kMaxStepWarpsReg : kMaxStepWarps))

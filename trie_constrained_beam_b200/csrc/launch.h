@@ -162,7 +162,4 @@ struct StepConfig {
   int smem_bytes;
 };
 
-bool choose_step_config(int V, int esize, int extra_bytes, int prefix_words, int n, bool reg,
-                        StepConfig* cfg);
-
 }  // namespace sidbeam
