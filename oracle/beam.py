@@ -118,12 +118,16 @@ def beam_finalize(bp_parent, bp_code, last_score, last_node):
     return {"sids": sids, "leaf": leaf, "score": score}
 
 
-def beam_search(trie, R: int, n: int, depth: int, V: int, logits_for_rows):
+def beam_search(trie, R: int, n: int, depth: int, V: int, logits_for_rows, widths=None):
     """Full constrained beam search from the root.
 
     logits_for_rows(step, prefixes, requests) -> logits [rows, V] for the given
     live prefixes (int array [rows, step]) of the given requests (int array
     [rows]); dead rows are never asked for.
+    widths: optional beams per request (each <= n): after every step request r
+    keeps its widths[r] best and the rest of its n slots become padding
+    (several requests of different widths sharing one step, flashrec 0.1.0,
+    Features > Decoding, "Scheduling").
     Returns finalize's dict plus per-step outputs (``steps``).
     """
     parent_scores = np.zeros(R)                    # step 0: one root row per request
@@ -140,6 +144,11 @@ def beam_search(trie, R: int, n: int, depth: int, V: int, logits_for_rows):
                 logits_for_rows(t, prefixes.reshape(R * B_in, t)[flat_live],
                                 flat_live // B_in))[:, :V]
         out = beam_step(trie, t, logits, parent_scores, parent_nodes, R, B_in, n, V)
+        if widths is not None:
+            for r, w in enumerate(widths):
+                out["score"][r, w:] = NEG_INF
+                for k in ("parent", "code", "node"):
+                    out[k][r, w:] = -1
         steps.append(out)
         new_prefixes = np.full((R, n, t + 1), -1, dtype=np.int64)
         for r in range(R):

@@ -401,6 +401,29 @@ def test_top_w_is_the_first_w_ranks_of_top_n():
             assert np.array_equal(wide[k][:, :w], narrow[k])
 
 
+def test_search_with_widths_equals_separate_searches():
+    """Requests of different widths in one search give, request by request, the
+    search of that request alone at its own width (padding past the width)."""
+    Vs = [8, 8, 8]
+    cat = host.draw_catalog(31, 300, Vs)
+    trie = oracle.OracleTrie(cat, Vs)
+    table = host.table_logits(31, 3, 3, 8, 1.5)
+
+    def fn_for(reqs_map):
+        def fn(step, prefixes, requests):
+            return np.stack([table[reqs_map[q], step] + 0.01 * prefixes.sum(axis=1)[i]
+                             for i, q in enumerate(requests)])
+        return fn
+
+    widths = [6, 2, 4]
+    res = oracle.beam_search(trie, 3, 6, 3, 8, fn_for([0, 1, 2]), widths=widths)
+    for r, w in enumerate(widths):
+        one = oracle.beam_search(trie, 1, w, 3, 8, fn_for([r]))
+        assert np.array_equal(res["sids"][r, :w], one["sids"][0])
+        assert np.array_equal(res["score"][r, :w], one["score"][0])
+        assert np.all(res["leaf"][r, w:] == -1)
+
+
 # ------------------------------------------------------------------ Gumbel top-k
 def test_oracle_philox_known_answers():
     """The oracle's own Philox4x32-10 against the published known-answer vectors."""
