@@ -137,6 +137,12 @@ def run_ours(args, world, rank, local):
     from sidgen.workloads import WORKLOADS
     from trie_constrained_beam_b200 import build as tbuild
 
+    # The oracle's tries and a pool of worker processes over all host cores,
+    # forked before the first CUDA call (a process forked after it cannot use
+    # the parent's CUDA state and can hang); workers inherit the tries.
+    pool = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pool = _start_oracle_pool(CFG, *(() if args.no_config_lines else (1, 2, 3)))
     torch.cuda.set_device(local)
     if rank == 0:
         tbuild.build()
@@ -292,11 +298,17 @@ def run_ours(args, world, rank, local):
     if not args.no_widths:
         widths = measure_widths(tcb, trie, w, base, dev)
 
+    configs = None
+    if not args.no_config_lines:
+        configs = {f"config{c}": measure_config(tcb, c, dev, pool, args.cpu_seconds / 3)
+                   for c in (1, 2, 3)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds, cat=cat)
+        cpu = cpu_baseline(w, base, search, live_rows, budget_s=args.cpu_seconds, pool=pool)
+    if pool is not None:
+        pool.terminate()
 
-    traffic = _profile_traffic()
+    traffic, traffic_kernel = _profile_traffic()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
@@ -304,6 +316,7 @@ def run_ours(args, world, rank, local):
         "config": _workload_config(w, {"parallelism": f"replicas x{world} (requests sharded)"}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     "traffic_kernel": traffic_kernel,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "kernel": "beam_step_kernel<bf16>, steady steps 1-4",
                      "bytes_per_launch": bytes_launch, "us_per_launch": dur_us},
@@ -317,6 +330,7 @@ def run_ours(args, world, rank, local):
         "fused_lmhead": fused,
         "gumbel_top_k": gumbel,
         "per_request_widths": widths,
+        "other_configs": configs,
         "cpu_baseline": cpu,
         "clocks": clk,
         "gpu_launches": K * (w.depth + 1),
@@ -503,18 +517,23 @@ def _n_leaves(cat):
 
 
 def _profile_traffic():
-    """DRAM bytes per steady beam_step launch from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "beam_step_wide_beam.md")
+    """DRAM bytes (read + write) per steady beam_step launch of the wide-beam
+    search, from the committed ncu record ``profiles/beam_step_wide_beam.json``
+    (written from the capture's raw counters), with the kernel name ncu printed
+    and the source of the build it measured. None when there is no record or
+    the record was taken on a different build of the kernel source."""
+    p = os.path.join(ROOT, "profiles", "beam_step_wide_beam.json")
     if not os.path.exists(p):
-        return None
-    for ln in open(p):
-        if ln.startswith("traffic_bytes_per_launch:"):
-            try:
-                v = ln.split(":", 1)[1].strip()
-                return None if v in ("", "null") else float(v)
-            except ValueError:
-                return None
-    return None
+        return None, None
+    rec = json.load(open(p))
+    src = os.path.join(ROOT, rec.get("source", ""))
+    if not os.path.exists(src):
+        return None, rec.get("kernel")
+    import hashlib
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec.get("source_sha256"):
+        return None, rec.get("kernel")
+    v = rec.get("traffic_bytes_per_launch")
+    return (None if v is None else float(v)), rec.get("kernel")
 
 
 # ----------------------------------------------------------------- oracle timing
@@ -531,29 +550,187 @@ def _oracle_trie(w, cat=None):
     return oracle.OracleTrie(w.catalog() if cat is None else cat, w.codes_per_level)
 
 
-def cpu_baseline(w, base, search, live_rows, budget_s=15.0, trie=None, cat=None):
-    """Time the oracle's beam step on a bounded sample of the same search: whole
-    requests (512 rows x 4,096 bf16 logits) of steps 1-4 in turn, until the
-    budget is spent, on this host's cores."""
+# Oracle tries of the workloads the pool serves (filled before the fork).
+_POOL_TRIES = {}
+
+
+def _host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def _start_oracle_pool(*cfgs):
+    import multiprocessing as mp
+
+    from sidgen.workloads import WORKLOADS
+    for c in cfgs:
+        if c not in _POOL_TRIES:
+            _POOL_TRIES[c] = _oracle_trie(WORKLOADS[c])
+    return mp.get_context("fork").Pool(os.cpu_count() or 1)
+
+
+def _oracle_task(job):
+    """One oracle beam step of one request (runs in a pool worker)."""
     import oracle
-    trie = trie or _oracle_trie(w, cat)
-    inputs = {t: _oracle_inputs(w, base, search, t) for t in range(1, w.depth)}
-    order = [(t, r) for r in range(w.R) for t in range(1, w.depth)]
-    done_rows = 0
-    calls = 0
-    t0 = time.perf_counter()
+    cfg, t, lg, ps, pn, B_in, n, V = job
+    oracle.beam_step(_POOL_TRIES[cfg], t, lg, ps, pn, 1, B_in, n, V)
+    return int(np.isfinite(ps).sum()) * V
+
+
+def _oracle_rates(cfg, jobs, budget_s, pool):
+    """Logits scored per second by the oracle: on one thread (in this process),
+    and on all cores (the pool, one request-step per task), each for about
+    budget_s seconds over the jobs in turn."""
+    import oracle
+    trie = _POOL_TRIES[cfg]
+    done, calls, t0 = 0, 0, time.perf_counter()
     while calls == 0 or time.perf_counter() - t0 < budget_s:
-        t, r = order[calls % len(order)]
-        lg, ps, pn, B_in = inputs[t]
-        sl = slice(r * B_in, (r + 1) * B_in)
-        oracle.beam_step(trie, t, lg[sl], ps[sl], pn[sl], 1, B_in, w.n, w.V)
-        done_rows += int(np.isfinite(ps[sl]).sum())
+        _, t, lg, ps, pn, B_in, n, V = jobs[calls % len(jobs)]
+        oracle.beam_step(trie, t, lg, ps, pn, 1, B_in, n, V)
+        done += int(np.isfinite(ps).sum()) * V
         calls += 1
-    el = time.perf_counter() - t0
-    return {"value": done_rows * w.V / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+    single = done / (time.perf_counter() - t0)
+    multi, mcalls = None, 0
+    if pool is not None:
+        per_call = (time.perf_counter() - t0) / calls
+        ncores = os.cpu_count() or 1
+        k = max(ncores, int(budget_s / per_call * ncores))
+        batch = [jobs[i % len(jobs)] for i in range(k)]
+        t1 = time.perf_counter()
+        mdone = sum(pool.imap_unordered(_oracle_task, batch))
+        multi = mdone / (time.perf_counter() - t1)
+        mcalls = k
+    return single, multi, calls, mcalls
+
+
+def _request_jobs(cfg, w, base, search, steps):
+    """Oracle inputs of whole requests (one request-step each) of the given steps."""
+    import torch
+    jobs = []
+    for t in steps:
+        lg = base[t].view(torch.int16).cpu().numpy().view(np.uint16) if base[t].dtype == torch.bfloat16 \
+            else base[t].cpu().numpy()
+        ps, pn, B_in = search.parents(t)
+        ps, pn = ps.cpu().numpy(), pn.cpu().numpy()
+        for r in range(w.R):
+            sl = slice(r * B_in, (r + 1) * B_in)
+            jobs.append((cfg, t, lg[sl], ps[sl], pn[sl], B_in, w.n, w.V))
+    return jobs
+
+
+def cpu_baseline(w, base, search, live_rows, budget_s=15.0, pool=None):
+    """The oracle's beam step timed on a bounded sample of the same search:
+    whole requests (512 rows x 4,096 bf16 logits) of steps 1-4 in turn, on one
+    host thread and on all host cores (one process per core, one request-step
+    per task)."""
+    jobs = _request_jobs(CFG, w, base, search, range(1, w.depth))
+    order = [jobs[(i % (w.depth - 1)) * w.R + (i // (w.depth - 1)) % w.R]
+             for i in range(len(jobs))]          # steps in turn, request by request
+    single, multi, calls, mcalls = _oracle_rates(CFG, order, budget_s, pool)
+    cores, model = _host_cpu()
+    line = {"value": single, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"oracle.beam_step on {calls} whole requests of steps 1-{w.depth - 1} "
-                      f"(512 rows x {w.V} bf16 logits each, steps in turn), {el:.1f} s, numpy "
-                      f"float64, single thread; host has {os.cpu_count()} cores"}
+                      f"(512 rows x {w.V} bf16 logits each, steps in turn), ~{budget_s:.0f} s, "
+                      f"numpy float64, one thread",
+            "host_cores": cores, "cpu_model": model}
+    if multi is not None:
+        line["all_cores"] = {"value": multi, "unit": UNIT, "cores": cores,
+                             "sample": f"{mcalls} request-steps of the same sample over a pool "
+                                       f"of {cores} processes"}
+    return line
+
+
+def measure_config(tcb, cfg, dev, pool, cpu_s):
+    """One workload's whole search on the device (the search's own logits,
+    resident in HBM, 3 rotating copies): per-step device times from events
+    inside a CUDA graph replay, the search time from graph replays, and (for
+    the HBM-bound flashrec-like workload) the steady steps' achieved HBM
+    bandwidth; plus the oracle on a bounded sample of the same search, on one
+    thread and on all cores."""
+    import torch
+    from sidgen import device as gdev
+    from sidgen import host
+    from sidgen.workloads import WORKLOADS
+
+    w = WORKLOADS[cfg]
+    cat = w.catalog()
+    trie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    search = tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    esize = 2 if w.dtype == "bf16" else 4
+    hashes = torch.from_numpy(host.request_roots(w.R).view(np.int64)).to(dev)
+    base, live_rows = [], []
+    for t in range(w.depth):
+        lg = torch.empty((search.rows(t), w.V), dtype=tdt, device=dev)
+        gdev.row_logits(w.logits_seed, hashes, w.V, w.sigma, lg)
+        ps, pn, B_in = search.parents(t)
+        live_rows.append(int(torch.isfinite(ps).sum().item()))
+        search.step(t, lg)
+        child = torch.empty((w.R * w.n,), dtype=torch.int64, device=dev)
+        gdev.child_hash(hashes, w.R, B_in, search.bp_parent[t], search.bp_code[t], w.n, t + 1,
+                        child)
+        hashes = child
+        base.append(lg)
+    search.finalize()
+    torch.cuda.synchronize()
+    ref = search.sids.clone()
+    sets = [base] + [[x.clone() for x in base] for _ in range(2)]
+    graphs = [search.capture(x) for x in sets]
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(w.depth + 2)]
+           for _ in sets]
+    egraphs = [search.capture(sets[i], events=evs[i]) for i in range(len(sets))]
+    for i in range(6):
+        graphs[i % 3].replay()
+    torch.cuda.synchronize()
+    reps = 60
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        graphs[i % 3].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us_search = e0.elapsed_time(e1) * 1e3 / reps
+    assert torch.equal(search.sids, ref)
+    acc = np.zeros(w.depth + 1)
+    for i in range(30):
+        egraphs[i % 3].replay()
+        torch.cuda.synchronize()
+        acc += [evs[i % 3][t].elapsed_time(evs[i % 3][t + 1]) for t in range(w.depth + 1)]
+    per = acc / 30 * 1e3
+    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+    logits = sum(r * w.V for r in live_rows)
+    out = {"workload": w.name, "us_per_search": us_search, "step_us": [float(x) for x in per[:-1]],
+           "finalize_us": float(per[-1]), "logits_per_s": logits / (us_search * 1e-6),
+           "timing": "CUDA graph replays of the whole search, 3 rotating logits copies; per-step "
+                     "times from events inside the graph"}
+    if cfg == 3:
+        steady = list(range(1, w.depth))
+        nbytes = [live_rows[t] * (w.V * esize + 8) + w.R * w.n * 16 for t in steady]
+        dur = float(np.mean([per[t] for t in steady]))
+        peak, kind = _peaks()
+        gbs = float(np.mean(nbytes)) / (dur * 1e-6) / 1e9
+        out["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                           "frac": gbs / peak, "bytes_per_launch": float(np.mean(nbytes)),
+                           "us_per_launch": dur, "peak_source": f"{kind} copy bandwidth"}
+    if pool is not None:
+        if cfg not in _POOL_TRIES:
+            return out
+        jobs = _request_jobs(cfg, w, base, search, range(1, w.depth))
+        single, multi, calls, mcalls = _oracle_rates(cfg, jobs, cpu_s, pool)
+        cores, model = _host_cpu()
+        out["cpu_baseline"] = {"unit": UNIT, "kind": "oracle", "one_thread": single,
+                               "all_cores": multi, "cores": cores, "cpu_model": model,
+                               "sample": f"{calls} request-steps of steps 1-{w.depth - 1} on one "
+                                         f"thread, {mcalls} on all cores"}
+    return out
 
 
 # ----------------------------------------------------------------- reference arm
@@ -626,7 +803,51 @@ def run_reference(args):
     }
 
 
+def record_traffic(csv_path, source):
+    """Write profiles/beam_step_wide_beam.json from an ncu CSV of the wide-beam
+    search's steady beam_step launches (steps 1-4), taken with
+    --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+    --csv: DRAM bytes read + written per launch (mean over the launches), the
+    kernel name as ncu printed it, and the sha256 of the kernel source it
+    measured (bench.py reports the traffic only while that source is unchanged)."""
+    import csv
+    import hashlib
+    rows = [r for r in csv.reader(open(csv_path)) if r]
+    hdr_i = next(i for i, r in enumerate(rows) if "Metric Name" in r)
+    hdr = rows[hdr_i]
+    col = {h: i for i, h in enumerate(hdr)}
+    per = {}
+    names = {}
+    for r in rows[hdr_i + 1:]:
+        if len(r) != len(hdr):
+            continue
+        lid = r[col["ID"]]
+        m, v, u = r[col["Metric Name"]], r[col["Metric Value"]].replace(",", ""), r[col["Metric Unit"]]
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-3,
+                 "usecond": 1, "msecond": 1e3}.get(u, 1)
+        per.setdefault(lid, {})[m] = float(v) * scale
+        names[lid] = r[col["Kernel Name"]]
+    launches = [d for d in per.values() if "dram__bytes_read.sum" in d]
+    traffic = [d["dram__bytes_read.sum"] + d.get("dram__bytes_write.sum", 0.0) for d in launches]
+    rec = {"kernel": sorted(set(names.values())),
+           "launches": len(launches),
+           "traffic_bytes_per_launch": float(np.mean(traffic)),
+           "traffic_bytes_each": traffic,
+           "gpu_time_us_each": [d.get("gpu__time_duration.sum") for d in launches],
+           "source": source,
+           "source_sha256": hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest(),
+           "how": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                  "--clock-control none -k regex:beam_ -s 1 -c 4 --csv on bench.py (the steady "
+                  "steps 1-4 of the generating wide-beam search); cold-cache, serialised launches"}
+    out = os.path.join(ROOT, "profiles", "beam_step_wide_beam.json")
+    json.dump(rec, open(out, "w"), indent=1)
+    print(out, rec["traffic_bytes_per_launch"])
+
+
 def main():
+    if len(sys.argv) >= 2 and sys.argv[1] == "--record-traffic":
+        record_traffic(sys.argv[2], sys.argv[3])
+        return
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
@@ -645,10 +866,18 @@ def main():
     ap.add_argument("--no-catalog", action="store_true",
                     help="skip the catalog_score_topk throughput lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-config-lines", action="store_true",
+                    help="skip the whole-search lines of the tiny, SPRINT-like and "
+                         "flashrec-like workloads (configs 1-3)")
     ap.add_argument("--copies", type=int, default=COPIES,
                     help="rotating copies of the per-step logits (3 keeps reads out of L2)")
     args = ap.parse_args()
     world, rank, local = _dist()
+    if args.gpus != world:
+        # One process per GPU: N GPUs means N ranks launched by torch.distributed.run.
+        print(json.dumps({"error": f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch "
+                                   f"{args.gpus} ranks with torch.distributed.run"}), flush=True)
+        sys.exit(2)
 
     if args.impl == "reference":
         if rank == 0:

@@ -132,10 +132,12 @@ def to_host_logits(logits, V):
     return x.cpu().numpy()
 
 
-def oracle_search_with_gaps(trie, R, n, depth, V, seed, sigma, dtype):
+def oracle_search_with_gaps(trie, R, n, depth, V, seed, sigma, dtype, widths=None):
     """Oracle search (host generator) that also reports, per request, the smallest
     gap over steps between the n-th and the (n+1)-th candidate: a near-tie there
-    changes the beam set, so end-to-end parity is only defined where it is wide."""
+    changes the beam set, so end-to-end parity is only defined where it is wide.
+    widths: beams kept per request (each <= n); the gap is then the one at the
+    request's own width, and slots past it are padding (as oracle.beam_search)."""
     def fn(step, prefixes, requests):
         return host.row_logits(seed, host.prefix_hashes(prefixes, requests), V, sigma,
                                dtype=dtype)
@@ -154,10 +156,16 @@ def oracle_search_with_gaps(trie, R, n, depth, V, seed, sigma, dtype):
             z[live] = _widen(fn(t, flat[live], live // B_in))
         ext = oracle.beam_step(trie, t, z, scores, nodes, R, B_in, n + 1, V)
         sc = ext["score"]
-        for r in range(R):   # boundary gap: n-th kept vs first left out
-            if np.isfinite(sc[r, n]):
-                min_gap[r] = min(min_gap[r], float(sc[r, n - 1] - sc[r, n]))
-        out = {k: v[:, :n] for k, v in ext.items()}
+        for r in range(R):   # boundary gap: the last kept vs the first left out
+            wr = n if widths is None else int(widths[r])
+            if wr > 0 and np.isfinite(sc[r, wr]):
+                min_gap[r] = min(min_gap[r], float(sc[r, wr - 1] - sc[r, wr]))
+        out = {k: v[:, :n].copy() for k, v in ext.items()}
+        if widths is not None:
+            for r, wr in enumerate(widths):
+                out["score"][r, wr:] = -np.inf
+                for k in ("parent", "code", "node"):
+                    out[k][r, wr:] = -1
         outs.append(out)
         bpp.append(out["parent"])
         bpc.append(out["code"])

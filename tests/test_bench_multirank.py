@@ -65,3 +65,13 @@ def test_reference_arm_runs_on_rank_zero_only():
                          capture_output=True, text=True, env=env, timeout=120, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip() == ""
+
+
+def test_gpus_flag_must_match_the_launched_ranks():
+    """--gpus N without N launched ranks is an error, not a silent 1-GPU run."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "8",
+                          "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, env=env, timeout=120, cwd=ROOT)
+    assert out.returncode != 0
+    assert "WORLD_SIZE is 1" in out.stdout

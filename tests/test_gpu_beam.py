@@ -96,6 +96,36 @@ def test_step_local_parity_padded_ld_and_fp32_config3_shape(tcb):
 
 
 # ---------------------------------------------------------------- end to end
+def _compare_search(otrie, w, R, sids, leaf, scores, ref):
+    """End-to-end rule: every beam a catalog SID with its leaf id, scores within
+    depth x TOL, and SIDs identical at every rank with wide gaps on both sides,
+    for the requests whose beam boundary never had a near-tie. Returns the
+    number of requests compared rank by rank."""
+    sids, leaf, scores = _host(sids), _host(leaf), _host(scores).astype(np.float64)
+    catalog = {tuple(s) for s in otrie.leaves.tolist()}
+    compared = 0
+    for r in range(R):
+        # Every GPU beam is a catalog SID (invalid rate 0) and its leaf id matches.
+        for k in range(leaf.shape[1]):
+            if leaf[r, k] >= 0:
+                assert tuple(sids[r, k]) in catalog
+                assert tuple(otrie.leaves[leaf[r, k]]) == tuple(sids[r, k])
+        np.testing.assert_allclose(scores[r], ref["score"][r], atol=TOL * w.depth, rtol=0)
+        if ref["min_gap"][r] > 10 * TOL * w.depth:
+            os_ = ref["score"][r]
+            n = os_.shape[0]
+            for k in range(n):
+                if not np.isfinite(os_[k]):
+                    break  # padding
+                lo = k == 0 or os_[k - 1] - os_[k] > TOL * w.depth
+                hi = k == n - 1 or not np.isfinite(os_[k + 1]) or os_[k] - os_[k + 1] > TOL * w.depth
+                if lo and hi:
+                    assert np.array_equal(sids[r, k], ref["sids"][r, k])
+                    assert leaf[r, k] == ref["leaf"][r, k]
+            compared += 1
+    return compared
+
+
 @pytest.mark.parametrize("cfg", [1, 2])
 def test_end_to_end_parity(tcb, cfg):
     w = WORKLOADS[cfg]
@@ -104,26 +134,24 @@ def test_end_to_end_parity(tcb, cfg):
     _, sids, leaf, scores = run_gpu_search(gtrie, w.R, w.n, w.depth, w.V, w.logits_seed, w.sigma,
                                            w.dtype)
     ref = oracle_search_with_gaps(otrie, w.R, w.n, w.depth, w.V, w.logits_seed, w.sigma, w.dtype)
-    sids, leaf, scores = _host(sids), _host(leaf), _host(scores).astype(np.float64)
-    catalog = {tuple(s) for s in otrie.leaves.tolist()}
-    compared = 0
-    for r in range(w.R):
-        # Every GPU beam is a catalog SID (invalid rate 0) and its leaf id matches.
-        for k in range(w.n):
-            if leaf[r, k] >= 0:
-                assert tuple(sids[r, k]) in catalog
-                assert tuple(otrie.leaves[leaf[r, k]]) == tuple(sids[r, k])
-        np.testing.assert_allclose(scores[r], ref["score"][r], atol=TOL * w.depth, rtol=0)
-        if ref["min_gap"][r] > 10 * TOL * w.depth:
-            os_ = ref["score"][r]
-            for k in range(w.n):
-                lo = k == 0 or os_[k - 1] - os_[k] > TOL * w.depth
-                hi = k == w.n - 1 or os_[k] - os_[k + 1] > TOL * w.depth
-                if lo and hi:
-                    assert np.array_equal(sids[r, k], ref["sids"][r, k])
-                    assert leaf[r, k] == ref["leaf"][r, k]
-            compared += 1
-    assert compared >= w.R // 2
+    assert _compare_search(otrie, w, w.R, sids, leaf, scores, ref) >= w.R // 2
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_end_to_end_parity_full_beam_sampled_requests(tcb, cfg):
+    """The flashrec-like (64 x 128, V = 8192, 1M SIDs, CSR) and wide-beam (16 x
+    512, V = 4096, 8M SIDs, dense levels 1-2 and CSR below) workloads at their
+    full beam width and depth, for the first two requests: the chained steps,
+    the dense-to-CSR level switch, the back-pointers and finalize against the
+    oracle's whole search."""
+    w = WORKLOADS[cfg]
+    cat, otrie = _catalog(cfg)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    R = 2
+    _, sids, leaf, scores = run_gpu_search(gtrie, R, w.n, w.depth, w.V, w.logits_seed, w.sigma,
+                                           w.dtype)
+    ref = oracle_search_with_gaps(otrie, R, w.n, w.depth, w.V, w.logits_seed, w.sigma, w.dtype)
+    _compare_search(otrie, w, R, sids, leaf, scores, ref)
 
 
 def test_exhaustive_beam_equals_brute_force(tcb):
@@ -488,3 +516,26 @@ def test_per_request_widths_equal_separate_searches(tcb):
         assert np.array_equal(scores[r, :wr].view(np.uint32), c1[0].view(np.uint32))
         assert np.all(leaf[r, wr:] == -1) and np.all(sids[r, wr:] == -1)
         assert np.all(np.isneginf(scores[r, wr:]))
+
+
+def test_per_request_widths_match_oracle(tcb):
+    """Requests of widths 64, 17, 1 and 40 sharing every launch (eager calls and
+    the captured graph of the whole search, which must agree bit for bit)
+    against the oracle's search with the same per-request widths (flashrec
+    0.1.0, Features > Decoding, "Scheduling"), under the end-to-end rule."""
+    w = WORKLOADS[2]
+    cat, otrie = _catalog(2)
+    gtrie = tcb.sid_trie_build(cat, w.codes_per_level, w.layouts)
+    widths = [64, 17, 1, 40]
+    n = max(widths)
+    R = len(widths)
+    sids, leaf, scores = _search_roots(tcb, gtrie, host.request_roots(R), n, w.depth, w.V,
+                                       w.logits_seed, w.sigma, widths=widths, graph=True)
+    ref = oracle_search_with_gaps(otrie, R, n, w.depth, w.V, w.logits_seed, w.sigma, w.dtype,
+                                  widths=widths)
+    import torch
+    compared = _compare_search(otrie, w, R, torch.from_numpy(sids), torch.from_numpy(leaf),
+                               torch.from_numpy(scores), ref)
+    assert compared >= 2
+    for r, wr in enumerate(widths):
+        assert np.all(leaf[r, wr:] == -1) and np.all(np.isneginf(scores[r, wr:]))

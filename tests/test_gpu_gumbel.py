@@ -162,3 +162,26 @@ def test_gumbel_argument_checks(tcb):
     with pytest.raises(native.SidbeamError) as e:
         tcb.beam_step_gumbel(None, 0, z, ps, pn, 1, 4, 4, 8, 1.0, 1, o[0], o[1], o[2], o[3], small)
     assert e.value.status == native.SIDBEAM_ERR_WORKSPACE
+
+
+def test_gumbel_wide_beam_step1_shape(tcb):
+    """The wide-beam step-1 shape: 16 requests x 512 parent rows (8,192 rows),
+    V = 4,096 bf16 logits (sigma 3), a dense child bitmask over a catalog whose
+    two levels are Zipf(1.2) (so parents have from a few to thousands of
+    children), n = 512, T = 1: every request against the oracle."""
+    V, R, B_in, n, T = 4096, 16, 512, 512, 1.0
+    rng = np.random.default_rng(41)
+    cat = host.draw_catalog(4101, 300_000, [V, V], [("zipf", 1.2), ("zipf", 1.2)])
+    otrie = oracle.OracleTrie(cat, [V, V])
+    gtrie = tcb.sid_trie_build(cat, [V, V], [1, 1])
+    nodes = np.arange(otrie.n_nodes(1))
+    pn = np.concatenate([rng.choice(nodes, size=B_in, replace=False) for _ in range(R)])
+    pn = pn.astype(np.int32)
+    ps = np.concatenate([np.sort(rng.uniform(-9, -2, size=B_in))[::-1] for _ in range(R)])
+    ps = ps.astype(np.float32)
+    z = host.bf16_bits_to_f32(host.f32_to_bf16_bits(
+        (3.0 * rng.standard_normal((R * B_in, V))).astype(np.float32)))
+    seed = 0x5EED_0F_6B3E1
+    g = _run(tcb, gtrie, 1, z, ps, pn, R, B_in, n, V, T, seed, "bf16")
+    ref = oracle.beam_step_gumbel(otrie, 1, z, ps, pn, R, B_in, n, V, T, seed)
+    _compare(g, ref, R, n, T, otrie, 1, z, ps, pn, B_in, V, seed)

@@ -40,7 +40,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
                      cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
-                     float* row_lse, const int32_t* out_width);
+                     float* row_lse, const int32_t* out_width, size_t clear_bytes);
 
 namespace {
 
@@ -101,8 +101,10 @@ extern "C" int beam_step(const sidbeam_trie* trie, int step, const void* logits,
                       stream, 0u, nullptr);
 }
 
+namespace sidbeam {
+
 // The host checks every step entry point shares (shapes, pointers, alignment).
-static int check_step_args(const sidbeam_trie* trie, int step, const void* logits,
+int check_step_args(const sidbeam_trie* trie, int step, const void* logits,
                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
                            const float* out_scores, const int32_t* out_parent,
@@ -145,12 +147,15 @@ static int check_step_args(const sidbeam_trie* trie, int step, const void* logit
   return SIDBEAM_OK;
 }
 
-extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
-                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
-                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
-                            float* out_scores, int32_t* out_parent, int32_t* out_code,
-                            int32_t* out_node, void* workspace, size_t workspace_bytes,
-                            void* stream, unsigned flags, const int32_t* out_width) {
+// The deterministic step after every host check; clear_bytes > 0 zeroes the
+// head of the workspace on the stream right before the launch (after every
+// check, so that a rejected call enqueues nothing).
+int beam_step_checked(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dtype dtype,
+                      int64_t ld, const float* parent_scores, const int32_t* parent_nodes, int R,
+                      int B_in, int n_out, int V, float* out_scores, int32_t* out_parent,
+                      int32_t* out_code, int32_t* out_node, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream, unsigned flags,
+                      const int32_t* out_width, size_t clear_bytes) {
   if (flags & ~static_cast<unsigned>(SIDBEAM_STEP_SKIP_ROWS))
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: unknown flags 0x%x", flags);
   const int rc = check_step_args(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R,
@@ -159,8 +164,22 @@ extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logi
   if (rc != SIDBEAM_OK) return rc;
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
-                          workspace_bytes, static_cast<cudaStream_t>(stream), flags, 0.f, 0ull,
-                          nullptr, out_width);
+                          workspace_bytes, stream, flags, 0.f, 0ull, nullptr, out_width,
+                          clear_bytes);
+}
+
+}  // namespace sidbeam
+
+extern "C" int beam_step_ex(const sidbeam_trie* trie, int step, const void* logits,
+                            sidbeam_dtype dtype, int64_t ld, const float* parent_scores,
+                            const int32_t* parent_nodes, int R, int B_in, int n_out, int V,
+                            float* out_scores, int32_t* out_parent, int32_t* out_code,
+                            int32_t* out_node, void* workspace, size_t workspace_bytes,
+                            void* stream, unsigned flags, const int32_t* out_width) {
+  return sidbeam::beam_step_checked(trie, step, logits, dtype, ld, parent_scores, parent_nodes,
+                                    R, B_in, n_out, V, out_scores, out_parent, out_code,
+                                    out_node, workspace, workspace_bytes,
+                                    static_cast<cudaStream_t>(stream), flags, out_width, 0);
 }
 
 // Gumbel steps keep every row's lse after the beam_step workspace.
@@ -200,7 +219,7 @@ extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* 
   return launch_beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
                           n_out, V, out_scores, out_parent, out_code, out_node, workspace,
                           workspace_bytes, static_cast<cudaStream_t>(stream), 0u, temperature,
-                          seed, row_lse, nullptr);
+                          seed, row_lse, nullptr, 0);
 }
 
 extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,

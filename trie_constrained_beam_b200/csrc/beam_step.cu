@@ -1524,7 +1524,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
                      int n_out, int V, float* out_scores, int32_t* out_parent, int32_t* out_code,
                      int32_t* out_node, void* workspace, size_t workspace_bytes,
                      cudaStream_t stream, unsigned flags, float gumbel_T, uint64_t gumbel_seed,
-                     float* row_lse, const int32_t* out_width) {
+                     float* row_lse, const int32_t* out_width, size_t clear_bytes) {
   StepArgs a{};
   a.logits = static_cast<const uint8_t*>(logits);
   a.bf16 = dtype == SIDBEAM_BF16;
@@ -1603,6 +1603,10 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaFuncSetAttribute");
   const dim3 grid(static_cast<unsigned>(a.part.grid));
   const dim3 block(static_cast<unsigned>(32 * a.cfg.W));
+  if (clear_bytes) {  // every check has passed: the caller's counters start at zero
+    e = cudaMemsetAsync(workspace, 0, clear_bytes, stream);
+    if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaMemsetAsync");
+  }
   switch (which) {
     case 0: beam_step_kernel<0, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 1: beam_step_kernel<1, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;

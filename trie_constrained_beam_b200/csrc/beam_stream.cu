@@ -331,17 +331,24 @@ __device__ __forceinline__ float finite_or_ninf(float x) {
 // child score is at most its parent's), the same in every CTA. Two slots
 // alternate so that one can be cleared while the other is read. All
 // consumer threads call it.
-__device__ __forceinline__ float segment_ref(const SArgs& a, const Team& t, SelCtl* ctl, int r,
-                                             int slot) {
+// This thread's part of the maximum (loads only; combined by segment_ref_finish).
+__device__ __forceinline__ float segment_ref_part(const SArgs& a, const Team& t, int r) {
   float m = __int_as_float(0xFF800000);
   const float* ps = a.parent_scores + static_cast<int64_t>(r) * a.B_in;
   for (int i = t.tid; i < a.B_in; i += t.T) m = fmaxf(m, finite_or_ninf(ps[i]));
+  return m;
+}
+__device__ __forceinline__ float segment_ref_finish(const Team& t, SelCtl* ctl, int slot, float m) {
   m = warp_max(m);
   if (t.lane == 0 && m > __int_as_float(0xFF800000)) atomicMax(&ctl->ref_ord[slot], ord_f32(m));
   team_sync(t);
   const unsigned o = *reinterpret_cast<volatile unsigned*>(&ctl->ref_ord[slot]);
   if (t.tid == 0) ctl->ref_ord[slot ^ 1] = 0u;
   return o ? unord_f32(o) : 0.f;
+}
+__device__ __forceinline__ float segment_ref(const SArgs& a, const Team& t, SelCtl* ctl, int r,
+                                             int slot) {
+  return segment_ref_finish(t, ctl, slot, segment_ref_part(a, t, r));
 }
 
 // End of the segment of request r (all consumer warps, in the same order).
@@ -380,6 +387,7 @@ __device__ __noinline__ bool segment_end(const SArgs& a, Team team, WarpBuf wb, 
   f.direct_vals =
       last ? reinterpret_cast<int32_t*>(stages + static_cast<size_t>(direct_cap) * 8) : nullptr;
   f.direct_cap = last ? direct_cap : 0;
+  f.read_request_bound = 0;  // the warps fold the request's bound in row by row
   const StepOut out{a.out_scores, a.out_parent, a.out_code, a.out_node,
                     a.n, static_cast<uint32_t>(a.V), a.out_width};
   return segment_flush(team, wb, ctl, f, out);
@@ -576,7 +584,13 @@ __global__ void __launch_bounds__(kStreamMaxWarps * 32, 1)
     cp_async_commit();
   }
   // 2. Parent data, 32 rows at a time (lane k: row base + k), then the trie
-  //    data of the first rows.
+  //    data of the first rows; the first segment's histogram reference (the
+  //    request's largest parent score) is loaded alongside.
+  int64_t lo, hi;
+  a.part.range(static_cast<int>(blockIdx.x), lo, hi);
+  const int r_first = static_cast<int>(lo / a.B_in);
+  const int r_last = static_cast<int>((hi - 1) / a.B_in);
+  const float mref = segment_ref_part(a, team, r_first);
   int mbase = 0;
   uint4 mb = make_uint4(0xFF800000u, 0u, 0u, 0u);
   if (lane < q.count) mb = row_meta(a, q.row(lane));
@@ -590,12 +604,8 @@ __global__ void __launch_bounds__(kStreamMaxWarps * 32, 1)
 
   WarpBuf wb{wkeys + static_cast<size_t>(warp) * p.Cw, wvals + static_cast<size_t>(warp) * p.Cw,
              whist + warp * 256, p.Cw, 0, 0ull, 0};
-  int64_t lo, hi;
-  a.part.range(static_cast<int>(blockIdx.x), lo, hi);
-  const int r_first = static_cast<int>(lo / a.B_in);
-  const int r_last = static_cast<int>((hi - 1) / a.B_in);
   int ref_slot = 0;
-  float C = segment_ref(a, team, ctl, r_first, ref_slot);
+  float C = segment_ref_finish(team, ctl, ref_slot, mref);
   int cur_r = r_first;
   int64_t seg_end = static_cast<int64_t>(cur_r + 1) * a.B_in;
   const uint4 ninf = BF16 ? make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u)
@@ -726,6 +736,7 @@ __global__ void __launch_bounds__(kStreamMaxWarps * 32, 1)
         const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
         if (c > wb.thr) wb.thr = c;
         if (req > wb.thr) wb.thr = req;
+        if (req > c && lane == 0) atomicMax(&ctl->cta_thr, req);  // the CTA's bound holds it too
       }
       float zthr = zthreshold(wb.thr, s, lse);
       bool binned_any = false;
@@ -849,24 +860,44 @@ __global__ void __launch_bounds__(kStreamMaxWarps * 32, 1)
               zthr = zthreshold(wb.thr, s, lse);
             }
           };
-          // Few hits: count and offer in one pass. Many: count them all,
-          // raise the threshold from this CTA's histogram, and offer only
-          // the hits that still reach it.
-          int mode = nh <= kOnePassHits ? 0 : 1;
-          const uint32_t h0 = hp[0], h1 = hp[1], h2 = hp[2], h3 = hp[3];
-          for (;;) {
-            walk(mode);
-            if (mode != 1) break;
-            hp[0] = h0;
-            hp[1] = h1;
-            hp[2] = h2;
-            hp[3] = h3;
+          // Few hits: count and offer in one walk. Many: count them all lane
+          // by lane (no votes: every lane bins its own hits), raise the
+          // threshold from this CTA's histogram, keep only the hits that
+          // still reach it, and offer those.
+          if (nh <= kOnePassHits) {
+            walk(0);
+          } else {
+#pragma unroll
+            for (int i = 0; i < kRegVecs; ++i) {
+              if (!full_chunk && 32 * i >= nvec) continue;
+              const unsigned bits = (hp[i >> 2] >> ((i & 3) * 8)) & 0xFFu;
+              if (bits) {
+#pragma unroll 1
+                for (int e = 0; e < kPerVec; ++e)
+                  if ((bits >> e) & 1u)
+                    atomicAdd(&ctl->hist[score_bin(s + (vec_elem<BF16>(x[i], e) - lse), C)], 1u);
+              }
+            }
+            wb.binned += nh;
+            if (lane == 0) atomicAdd(&ctl->hist_total, static_cast<unsigned>(nh));
             __syncwarp();
             wb.binned = kRefreshAfter;  // rescan this CTA's histogram now (inline: no call)
             refresh_thr(wb, ctl, static_cast<uint32_t>(a.n), C, lane, sinks);
             const float z1 = zthreshold(wb.thr, s, lse);
             if (z1 > zthr) zthr = z1;
-            mode = 2;
+#pragma unroll
+            for (int i = 0; i < kRegVecs; ++i) {
+              if (!full_chunk && 32 * i >= nvec) continue;
+              const unsigned bits = (hp[i >> 2] >> ((i & 3) * 8)) & 0xFFu;
+              unsigned keep = 0u;
+              if (bits) {
+#pragma unroll 1
+                for (int e = 0; e < kPerVec; ++e)
+                  if (((bits >> e) & 1u) && vec_elem<BF16>(x[i], e) >= zthr) keep |= 1u << e;
+              }
+              hp[i >> 2] = (hp[i >> 2] & ~(0xFFu << ((i & 3) * 8))) | (keep << ((i & 3) * 8));
+            }
+            walk(2);
           }
           binned_any = true;
         }

@@ -51,6 +51,16 @@ int set_error(int status, const char* fmt, ...);
 int cuda_error(cudaError_t e, const char* what);
 int device_sm_count();
 
+// The deterministic step behind every host check of beam_step_ex; with
+// clear_bytes > 0 the first clear_bytes of the workspace are zeroed on the
+// stream right before the launch (nothing is enqueued when a check fails).
+int beam_step_checked(const sidbeam_trie* trie, int step, const void* logits, sidbeam_dtype dtype,
+                      int64_t ld, const float* parent_scores, const int32_t* parent_nodes, int R,
+                      int B_in, int n_out, int V, float* out_scores, int32_t* out_parent,
+                      int32_t* out_code, int32_t* out_node, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream, unsigned flags,
+                      const int32_t* out_width, size_t clear_bytes);
+
 // CSR nodes with more children than this also get a bitmask row (the step
 // kernel handles up to this many children of a node one per lane).
 constexpr int kListMaxChildren = 32;

@@ -73,14 +73,13 @@ extern "C" int beam_step_noalloc(const sidbeam_trie* trie, int step, const void*
   const int rc = scratch_address(&scratch);
   if (rc != SIDBEAM_OK) return rc;
   // The counters at the head of the scratch must start at zero (status word,
-  // per-request tickets and bounds, partial-list sizes); clear them on the
-  // stream so the call does not depend on what an earlier call left behind.
+  // per-request tickets and bounds, histograms, partial-list sizes); the step
+  // clears them on the stream after all of its argument checks have passed,
+  // right before its kernel, so a rejected call enqueues nothing.
   const Partition p = make_partition(R, B_in, std::min(device_sm_count(), 640));
   const WorkspaceLayout ws = workspace_layout(R, p.maxG, n_out);
-  const cudaError_t e =
-      cudaMemsetAsync(scratch, 0, ws.part_keys, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_error(e, "beam_step_noalloc: cudaMemsetAsync");
-  return beam_step(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in, n_out, V,
-                   out_scores, out_parent, out_code, out_node, scratch,
-                   SIDBEAM_NOALLOC_SCRATCH_BYTES, stream);
+  return beam_step_checked(trie, step, logits, dtype, ld, parent_scores, parent_nodes, R, B_in,
+                           n_out, V, out_scores, out_parent, out_code, out_node, scratch,
+                           SIDBEAM_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream), 0u,
+                           nullptr, ws.part_keys);
 }
