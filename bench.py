@@ -35,6 +35,8 @@ METRIC = "beam-step logits scored/sec & achieved HBM GB/s (% of B200 peak) at be
 UNIT = "logits/s"
 CFG = 4
 COPIES = 3
+SM_COUNT = 148      # B200 streaming multiprocessors
+SM_MAX_MHZ = 1965   # clocks.max.sm of the B200s measured here
 
 
 def _peaks():
@@ -375,6 +377,15 @@ def measure_catalog(tcb, trie4, cat4, w4, dev):
         assert tcb.sidbeam_get_device_status(ws) == 0
         out = {"us_per_call": us, "pairs_per_s": R * n_leaves / (us * 1e-6),
                "requests": R, "sids": n_leaves, "depth": L, "codes_per_level": V, "K": K}
+        # Roofline: every (request, SID, level) is one 4-byte shared-memory table
+        # lookup; the pipe serves one word per lane per clock on each SM.
+        lookups = float(R) * n_leaves * L
+        peak = SM_COUNT * 32 * SM_MAX_MHZ * 1e6
+        out["roofline"] = {"bound": "alu", "unit": "lookups/s", "achieved": lookups / (us * 1e-6),
+                           "peak": peak, "frac": lookups / (us * 1e-6) / peak,
+                           "peak_source": f"{SM_COUNT} SMs x 32 lanes x {SM_MAX_MHZ} MHz "
+                                          "(one shared-memory word per lane per clock)",
+                           "code_bytes": n_leaves * L * 2, "table_bytes": R * L * V * 4}
         if sim is not None:
             out["similarity_dim"] = int(sim[0].shape[1])
         return out
@@ -824,7 +835,7 @@ def record_traffic(csv_path, source):
         lid = r[col["ID"]]
         m, v, u = r[col["Metric Name"]], r[col["Metric Value"]].replace(",", ""), r[col["Metric Unit"]]
         scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-3,
-                 "usecond": 1, "msecond": 1e3}.get(u, 1)
+                 "ns": 1e-3, "usecond": 1, "us": 1, "msecond": 1e3, "ms": 1e3}.get(u, 1)
         per.setdefault(lid, {})[m] = float(v) * scale
         names[lid] = r[col["Kernel Name"]]
     launches = [d for d in per.values() if "dram__bytes_read.sum" in d]
@@ -837,8 +848,10 @@ def record_traffic(csv_path, source):
            "source": source,
            "source_sha256": hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest(),
            "how": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
-                  "--clock-control none -k regex:beam_ -s 1 -c 4 --csv on bench.py (the steady "
-                  "steps 1-4 of the generating wide-beam search); cold-cache, serialised launches"}
+                  "--clock-control none -k regex:beam_step_kernel -s 1 -c 4 --csv on python "
+                  "bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --copies 1 --no-fused "
+                  "--no-catalog --no-gumbel --no-widths --no-config-lines (the steady steps 1-4 "
+                  "of the generating wide-beam search); cold-cache, serialised launches"}
     out = os.path.join(ROOT, "profiles", "beam_step_wide_beam.json")
     json.dump(rec, open(out, "w"), indent=1)
     print(out, rec["traffic_bytes_per_launch"])
