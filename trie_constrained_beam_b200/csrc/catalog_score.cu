@@ -13,8 +13,10 @@
 //
 // (request, leaf) pairs are laid out request-major and split evenly over the
 // CTAs, exactly like beam rows in beam_step. A CTA keeps the current
-// request's table in shared memory, each warp scores 32 leaves at a time from
-// the SoA leaf codes (coalesced uint16 loads), and candidates go through the
+// request's table in shared memory. Token sums: each lane scores 8
+// consecutive leaves at a time (one 16-byte load of their codes per level, all
+// levels' loads in flight before the first lookup), a warp 256; with the
+// similarity term a lane scores one leaf at a time. Candidates go through the
 // same warp / CTA / request top-n machinery as beam_step (topn.cuh).
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,6 +34,8 @@ namespace {
 using namespace dev;
 
 constexpr int kScoreWarps = 8;
+constexpr int kLeavesPerLane = 8;  // token sums: consecutive leaves per lane (one 16-byte code load)
+constexpr int kLevelBatch = 6;     // levels whose code loads are issued before the lookups
 
 struct ScoreConfig {
   int W, Cw, ctas_per_sm;
@@ -39,7 +43,7 @@ struct ScoreConfig {
 };
 
 struct ScoreArgs {
-  const uint16_t* leaf_codes;  // [depth][stride]
+  const uint16_t* leaf_codes;  // [depth][stride], stride a multiple of 8, zero past N
   int64_t stride;
   int64_t N;
   int depth;
@@ -149,7 +153,93 @@ __global__ void __launch_bounds__(kScoreWarps * 32, 2)
     const int64_t j_lo = seg_lo - static_cast<int64_t>(r) * a.N;
     const int64_t j_hi = seg_hi - static_cast<int64_t>(r) * a.N;
     int batches = 0;
-    for (int64_t j0 = j_lo + static_cast<int64_t>(warp) * 32; j0 < j_hi;
+    if constexpr (!SIM) {
+      // Lane: leaves jv .. jv+7 (jv a multiple of 8; those outside [j_lo, j_hi)
+      // are computed from the zero padding or a neighbour's codes and dropped).
+      constexpr int E = kLeavesPerLane;
+      const int64_t jstart = j_lo & ~static_cast<int64_t>(E - 1);
+      // Up to kLevelBatch levels: the next block's codes are loaded while this
+      // block's lookups run (software pipelining, one block ahead).
+      const bool pf = a.depth <= kLevelBatch;
+      uint4 qn[kLevelBatch];
+      if (pf) {
+        const int64_t jv0 =
+            jstart + static_cast<int64_t>(warp) * 32 * E + static_cast<int64_t>(E) * lane;
+#pragma unroll
+        for (int u = 0; u < kLevelBatch; ++u) {
+          qn[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (jv0 < j_hi && u < a.depth)
+            qn[u] = __ldg(reinterpret_cast<const uint4*>(
+                a.leaf_codes + static_cast<int64_t>(u) * a.stride + jv0));
+        }
+      }
+      for (int64_t jb = jstart + static_cast<int64_t>(warp) * 32 * E; jb < j_hi;
+           jb += static_cast<int64_t>(cfg.W) * 32 * E) {
+        const int64_t jv = jb + static_cast<int64_t>(E) * lane;
+        const bool any_in = jv < j_hi;
+        float sc[E];
+        for (int l0 = 0; l0 < a.depth; l0 += kLevelBatch) {
+          uint4 q[kLevelBatch];
+          if (l0 == 0 && pf) {
+#pragma unroll
+            for (int u = 0; u < kLevelBatch; ++u) q[u] = qn[u];
+          } else {
+#pragma unroll
+            for (int u = 0; u < kLevelBatch; ++u) {
+              q[u] = make_uint4(0u, 0u, 0u, 0u);
+              if (any_in && l0 + u < a.depth)
+                q[u] = __ldg(reinterpret_cast<const uint4*>(
+                    a.leaf_codes + static_cast<int64_t>(l0 + u) * a.stride + jv));
+            }
+          }
+          if (l0 == 0 && pf) {  // next iteration's codes in flight during these lookups
+            const int64_t jn = jv + static_cast<int64_t>(cfg.W) * 32 * E;
+#pragma unroll
+            for (int u = 0; u < kLevelBatch; ++u) {
+              qn[u] = make_uint4(0u, 0u, 0u, 0u);
+              if (jn < j_hi && u < a.depth)
+                qn[u] = __ldg(reinterpret_cast<const uint4*>(
+                    a.leaf_codes + static_cast<int64_t>(u) * a.stride + jn));
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kLevelBatch; ++u) {
+            if (l0 + u < a.depth) {
+              const float* tl = table + (l0 + u) * a.Vmax;
+              const uint32_t w4[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                const float v = tl[(w4[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu];
+                sc[e] = (l0 + u == 0) ? v : sc[e] + v;  // levels added in order
+              }
+            }
+          }
+        }
+        bool pass[E];
+        bool any = false;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int64_t j = jv + e;
+          pass[e] = j >= j_lo && j < j_hi &&
+                    make_key(sc[e], static_cast<uint32_t>(j)) >= wb.thr;
+          any |= pass[e];
+        }
+        if (!__any_sync(0xFFFFFFFFu, any)) continue;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint32_t j = static_cast<uint32_t>(jv + e);
+          const uint64_t key = make_key(sc[e], j);
+          const bool ok = pass[e] && key >= wb.thr;  // the threshold may have risen
+          if (!__any_sync(0xFFFFFFFFu, ok)) continue;
+          warp_bin(ctl->hist, ok, score_bin(sc[e], C), wb.binned, &ctl->hist_total);
+          if ((++batches & 7) == 0)
+            refresh_thr(wb, ctl, static_cast<uint32_t>(a.K), C, lane, sinks);
+          warp_offer(wb, ok, key, static_cast<int32_t>(j), static_cast<uint32_t>(a.K), lane,
+                     sinks);
+        }
+      }
+    }
+    for (int64_t j0 = j_lo + static_cast<int64_t>(warp) * 32; SIM && j0 < j_hi;
          j0 += static_cast<int64_t>(cfg.W) * 32) {
       const int64_t j = j0 + lane;
       const bool valid = j < j_hi;
@@ -224,7 +314,9 @@ bool choose_score_config(int depth, int Vmax, int K, int d, ScoreConfig* out) {
   static_assert(kScoreWarps * 256 >= 2 * dev::kHistBins, "rank-merge scratch lives in whist");
   int npow2 = 1;
   while (npow2 < K) npow2 <<= 1;
-  c.Cw = std::max(round_up(K, 32) + 512, round_up((npow2 + c.W - 1) / c.W, 32));
+  // Warp buffers: K plus 128 entries of slack between compactions (small
+  // enough that two CTAs of the wide-catalog shape share an SM).
+  c.Cw = std::max(round_up(K, 32) + 128, round_up((npow2 + c.W - 1) / c.W, 32));
   int o = 0;
   c.off_ctl = o;
   o += round_up(static_cast<int>(sizeof(SelCtl)), 128);

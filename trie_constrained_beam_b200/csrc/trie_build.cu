@@ -267,7 +267,9 @@ extern "C" int sid_trie_build(const int32_t* sids, int64_t n_sids, int depth,
   // 4. Leaf tables.
   {
     std::vector<int32_t> rows(leaf_row.begin(), leaf_row.end());
-    t->leaf_codes_stride = N + 8;
+    // Rows of a multiple of 8 codes (16-byte aligned), zero-padded past N: a
+    // scorer reads 8 consecutive leaves' codes with one 16-byte load.
+    t->leaf_codes_stride = (N + 7) / 8 * 8 + 8;
     std::vector<uint16_t> soa(static_cast<size_t>(depth) * t->leaf_codes_stride, 0);
     for (int64_t j = 0; j < N; ++j)
       for (int l = 0; l < depth; ++l)
