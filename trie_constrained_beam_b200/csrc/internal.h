@@ -22,11 +22,6 @@ struct StepTrie {
   int mask_words = 0;           // ceil(V / 32)
   int mask_stride = 0;          // mask_words rounded up to a multiple of 4 (16-byte rows)
   uint16_t* codes = nullptr;    // CSR: [P_{t+1} + 8]: code of child id q (padded for 16-B loads)
-  // CSR levels: nodes with more than kListMaxChildren children also get a
-  // V-bit child bitmask (row mask_idx[p] of `mask`, same row format as a
-  // dense level); mask_idx[p] = -1 for the others. Null when no node has one.
-  int32_t* mask_idx = nullptr;  // [P_t]
-  int64_t n_heavy = 0;          // rows of `mask` at a CSR level
   size_t bytes = 0;
 };
 
@@ -60,10 +55,6 @@ int beam_step_checked(const sidbeam_trie* trie, int step, const void* logits, si
                       int32_t* out_code, int32_t* out_node, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream, unsigned flags,
                       const int32_t* out_width, size_t clear_bytes);
-
-// CSR nodes with more children than this also get a bitmask row (the step
-// kernel handles up to this many children of a node one per lane).
-constexpr int kListMaxChildren = 32;
 
 // Device status word bits (first 4 bytes of a workspace).
 constexpr uint32_t kStatusBadNode = 1u;

@@ -5,9 +5,7 @@
 // nodes -> level-(t+1) codes) gets its own layout:
 //   dense: a V-bit child bitmask per node (rows padded to 16 bytes so one bulk
 //          copy moves a row) plus the first child id per node;
-//   CSR  : child id range per node plus the uint16 code of every child; nodes
-//          with many children also get a bitmask row (the step kernel then
-//          treats them like nodes of a dense level).
+//   CSR  : child id range per node plus the uint16 code of every child.
 // Node ids are lexicographic ranks of the distinct prefixes of each level, so
 // a node's children are consecutive ids in code order and leaf ids are the
 // ranks of the sorted unique SIDs.
@@ -210,48 +208,6 @@ extern "C" int sid_trie_build(const int32_t* sids, int64_t n_sids, int depth,
       st.bytes += words * 4;
     } else {
       const size_t nb = (static_cast<size_t>(st.n_child) + 8) * 2;
-      // Bitmask rows for the nodes with many children: the smallest fan-out
-      // limit (from kListMaxChildren up) whose rows stay within a budget of
-      // max(64 MiB, 4 x this level's CSR bytes).
-      const size_t row_bytes = static_cast<size_t>(st.mask_stride) * 4;
-      const size_t budget = std::max<size_t>(64u << 20, 4 * (nb + off_bytes));
-      std::vector<uint32_t> fan(static_cast<size_t>(st.n_parent));
-      for (int64_t p = 0; p < st.n_parent; ++p) fan[p] = off[p + 1] - off[p];
-      uint32_t limit = kListMaxChildren;
-      int64_t heavy = 0;
-      for (;;) {
-        heavy = 0;
-        for (int64_t p = 0; p < st.n_parent; ++p) heavy += fan[p] > limit ? 1 : 0;
-        if (static_cast<size_t>(heavy) * row_bytes <= budget || limit >= static_cast<uint32_t>(V))
-          break;
-        limit *= 2;
-      }
-      if (heavy > 0) {
-        std::vector<int32_t> idx(static_cast<size_t>(st.n_parent), -1);
-        std::vector<uint32_t> hm(static_cast<size_t>(heavy) * st.mask_stride, 0u);
-        int64_t h = 0;
-        for (int64_t p = 0; p < st.n_parent; ++p) {
-          if (fan[p] <= limit) continue;
-          idx[p] = static_cast<int32_t>(h);
-          for (uint32_t q = off[p]; q < off[p + 1]; ++q) {
-            const int c = child_code[q];
-            hm[static_cast<size_t>(h) * st.mask_stride + c / 32] |= 1u << (c % 32);
-          }
-          ++h;
-        }
-        if ((e = dev.alloc(&st.mask_idx, idx.size() * 4)) != cudaSuccess)
-          return cuda_error(e, "sid_trie_build");
-        if ((e = dev.alloc(&st.mask, hm.size() * 4)) != cudaSuccess)
-          return cuda_error(e, "sid_trie_build");
-        if ((e = cudaMemcpyAsync(st.mask_idx, idx.data(), idx.size() * 4, cudaMemcpyHostToDevice,
-                                 stream)) != cudaSuccess ||
-            (e = cudaMemcpyAsync(st.mask, hm.data(), hm.size() * 4, cudaMemcpyHostToDevice,
-                                 stream)) != cudaSuccess ||
-            (e = cudaStreamSynchronize(stream)) != cudaSuccess)
-          return cuda_error(e, "sid_trie_build");
-        st.n_heavy = heavy;
-        st.bytes += idx.size() * 4 + hm.size() * 4;
-      }
       child_code.resize(static_cast<size_t>(st.n_child) + 8, 0);
       if ((e = dev.alloc(&st.codes, nb)) != cudaSuccess) return cuda_error(e, "sid_trie_build");
       if ((e = cudaMemcpyAsync(st.codes, child_code.data(), nb, cudaMemcpyHostToDevice,
@@ -336,7 +292,6 @@ extern "C" void sid_trie_free(sidbeam_trie* t) {
     cudaFree(t->steps[l].off);
     cudaFree(t->steps[l].mask);
     cudaFree(t->steps[l].codes);
-    cudaFree(t->steps[l].mask_idx);
   }
   cudaFree(t->leaf_rows);
   cudaFree(t->leaf_codes);
