@@ -409,33 +409,42 @@ def measure_gumbel(tcb, trie, w, base, dev, reps=10):
     differ): per-step device times from events between eager launches, and
     logits scored per second over the whole search."""
     import torch
+
+    def steps_us(search):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(w.depth + 1)]
+
+        def once(record):
+            for t in range(w.depth):
+                if record:
+                    evs[t].record()
+                search.step(t, base[t])
+            if record:
+                evs[w.depth].record()
+
+        for _ in range(2):
+            once(False)
+        torch.cuda.synchronize()
+        per = np.zeros(w.depth)
+        for _ in range(reps):
+            once(True)
+            torch.cuda.synchronize()
+            per += [evs[t].elapsed_time(evs[t + 1]) * 1e3 for t in range(w.depth)]
+        assert tcb.sidbeam_get_device_status(search.workspace) == 0
+        return per / reps
+
     search = tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth, temperature=1.0,
                             seed=0x5EED_0F_6B3E1)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(w.depth + 1)]
-
-    def once(record):
-        for t in range(w.depth):
-            if record:
-                evs[t].record()
-            search.step(t, base[t])
-        if record:
-            evs[w.depth].record()
-
-    for _ in range(2):
-        once(False)
-    torch.cuda.synchronize()
-    per = np.zeros(w.depth)
-    for _ in range(reps):
-        once(True)
-        torch.cuda.synchronize()
-        per += [evs[t].elapsed_time(evs[t + 1]) * 1e3 for t in range(w.depth)]
-    per /= reps
-    assert tcb.sidbeam_get_device_status(search.workspace) == 0
+    per = steps_us(search)
+    det = steps_us(tcb.BeamSearch(trie, w.R, w.n, w.V, depth=w.depth))
     logits = sum(search.rows(t) * w.V for t in range(w.depth))
     return {"temperature": 1.0, "step_us": [float(x) for x in per],
+            "deterministic_step_us": [float(x) for x in det],
+            "ratio_to_deterministic": [float(x / y) for x, y in zip(per, det)],
             "logits_per_s": logits / (per.sum() * 1e-6),
-            "timing": "eager launches, events between steps, 10 searches",
-            "note": "Gumbel steps walk every row in shared memory (no register rows)"}
+            "timing": "eager launches, events between steps, 10 searches each (the "
+                      "deterministic search timed the same way on the same logits)",
+            "note": "rows of up to 8 KB in registers; one Philox draw per code that "
+                    "could reach the threshold"}
 
 
 def measure_widths(tcb, trie, w, base, dev, reps=50):

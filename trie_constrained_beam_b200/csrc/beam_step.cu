@@ -684,12 +684,25 @@ __device__ __forceinline__ void copy_row_regs(const uint8_t* zrow, int V, int la
 // (lane + 32k) whose code is a valid child with z >= zthr. Only vectors whose
 // largest logit reaches the threshold look at the mask. Returns whether any
 // lane of the warp has a hit.
-template <int BF16, bool FULL>
+// GUM: a hit is a candidate whose perturbed logit z + T*G reaches zthr; the
+// draw is made only for codes whose z + T*kGumbelMax does (r, b: the row's
+// request and parent slot, the draw's counter).
+template <int BF16, bool FULL, int GUM = 0>
 __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRegVecs], int nvec,
                                          float zthr, const uint32_t* wmask, int lane, int part,
-                                         int nparts, uint32_t (&hp)[kRegVecs / 4]) {
+                                         int nparts, uint32_t (&hp)[kRegVecs / 4], int r = 0,
+                                         uint32_t b = 0) {
   constexpr int kPerVec = BF16 ? 8 : 4;
   const bool dense = wmask != nullptr;
+  const float gm = GUM ? a.gumbel_T * kGumbelMax : 0.f;
+  auto hit = [&](float z, int code) -> bool {
+    if constexpr (GUM) return z + gm >= zthr && z + gumbel_noise(a, r, b, code) >= zthr;
+    return z >= zthr;
+  };
+  auto bulk = [&](float vmax) -> bool {  // may a code of the vector reach zthr?
+    if constexpr (GUM) return vmax + gm >= zthr;
+    return vmax >= zthr;
+  };
 #pragma unroll
   for (int i = 0; i < kRegVecs / 4; ++i) hp[i] = 0u;
   if (dense) {
@@ -709,12 +722,12 @@ __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRe
     Unrolled<kRegVecs>::run([&](auto kc) {
       constexpr int k = decltype(kc)::value;
       unsigned valid = vm[k];
-      if (valid && vec_max<BF16>(x[k]) >= zthr) {
+      if (valid && bulk(vec_max<BF16>(x[k]))) {
         unsigned bits = 0u;
         while (valid) {
           const int j = __ffs(valid) - 1;
           valid &= valid - 1u;
-          if (vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
+          if (hit(vec_elem<BF16>(x[k], j), (lane + 32 * k) * kPerVec + j)) bits |= 1u << j;
         }
         hp[k >> 2] |= bits << ((k & 3) * 8);
       }
@@ -724,14 +737,14 @@ __device__ __forceinline__ bool reg_hits(const StepArgs& a, const uint4 (&x)[kRe
       constexpr int k = decltype(kc)::value;
       const int v = lane + 32 * k;
       const bool mine = FULL || (32 * k < nvec && (k % nparts) == part && v < nvec);
-      if (mine && vec_max<BF16>(x[k]) >= zthr) {
+      if (mine && bulk(vec_max<BF16>(x[k]))) {
         const int cb = v * kPerVec;
         unsigned valid = (1u << kPerVec) - 1u;
         if (!FULL && a.V - cb < kPerVec) valid &= (1u << (a.V - cb)) - 1u;
         unsigned bits = 0u;
 #pragma unroll
         for (int j = 0; j < kPerVec; ++j)
-          if (((valid >> j) & 1u) && vec_elem<BF16>(x[k], j) >= zthr) bits |= 1u << j;
+          if (((valid >> j) & 1u) && hit(vec_elem<BF16>(x[k], j), cb + j)) bits |= 1u << j;
         hp[k >> 2] |= bits << ((k & 3) * 8);
       }
     });
@@ -756,7 +769,9 @@ struct TakeOut {
   int binned;
 };
 
-template <int BF16>
+// GUM: every hit's logit is perturbed by its own draw before it is tested and
+// keyed (the same draw as in reg_hits).
+template <int BF16, int GUM = 0>
 __device__ __noinline__ TakeOut take_hits(const StepArgs& a, const uint8_t* zrow, uint32_t h0,
                                           uint32_t h1, uint32_t h2, uint32_t h3,
                                           const uint32_t* wmask, uint32_t* wprefix, RowCtx c,
@@ -783,6 +798,11 @@ __device__ __noinline__ TakeOut take_hits(const StepArgs& a, const uint8_t* zrow
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) z[u] = code[u] >= 0 ? elem<BF16>(zrow, code[u]) : 0.f;
+    if constexpr (GUM) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (code[u] >= 0) z[u] += gumbel_noise(a, c.r, c.b, code[u]);
+    }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const bool has = code[u] >= 0 && (mode == kTakeBin || z[u] >= zthr);
@@ -1100,14 +1120,22 @@ __device__ __noinline__ bool segment_end(const StepArgs& a, Team team, WarpBuf w
 // and the request's first threshold. The scratch is not the segment
 // histogram, whose counts must match the candidates offered. Warp-collective;
 // zrow: the row's stage.
-template <int BF16>
+// GUM: the scores counted are the perturbed ones (each child's own draw; r, b:
+// the row's request and parent slot), so the bound holds for perturbed keys.
+template <int BF16, int GUM = 0>
 __device__ void seed_count(const StepArgs& a, const uint8_t* zrow, float s, float lse, uint32_t o0,
-                           uint32_t o1, float C, uint32_t* shist, int lane) {
+                           uint32_t o1, float C, uint32_t* shist, int lane, int r = 0,
+                           uint32_t b = 0) {
   constexpr int kPerVec = BF16 ? 8 : 4;
+  auto zeff = [&](float z, int code) -> float {
+    if constexpr (GUM) return z + gumbel_noise(a, r, b, code);
+    return z;
+  };
   if (a.layout == SIDBEAM_LAYOUT_CSR) {
     const uint32_t nst = csr_staged(a, o0, o1);
     for (uint32_t k = o0 + lane; k < o1; k += 32u) {
-      const float z = elem<BF16>(zrow, csr_code(a, zrow, o0, nst, k));
+      const int code = csr_code(a, zrow, o0, nst, k);
+      const float z = zeff(elem<BF16>(zrow, code), code);
       atomicAdd(&shist[score_bin(s + (z - lse), C)], 1u);
     }
     return;
@@ -1126,15 +1154,23 @@ __device__ void seed_count(const StepArgs& a, const uint8_t* zrow, float s, floa
 #pragma unroll
     for (int j = 0; j < kPerVec; ++j)
       if ((valid >> j) & 1u)
-        atomicAdd(&shist[score_bin(s + (vec_elem<BF16>(x, j) - lse), C)], 1u);
+        atomicAdd(&shist[score_bin(s + (zeff(vec_elem<BF16>(x, j), cb + j) - lse), C)], 1u);
   }
+}
+
+// The Gumbel count out of line (the draws' registers stay out of the kernel's
+// own allocation).
+template <int BF16>
+__device__ __noinline__ void seed_count_gumbel(const StepArgs& a, const uint8_t* zrow, float s,
+                                               float lse, uint32_t o0, uint32_t o1, float C,
+                                               uint32_t* shist, int lane, int r, uint32_t b) {
+  seed_count<BF16, 1>(a, zrow, s, lse, o0, o1, C, shist, lane, r, b);
 }
 
 // --------------------------------------------------------------- kernel
 template <int BF16, int REG, int GUM = 0>
 __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 32, 1)
     beam_step_kernel(const __grid_constant__ StepArgs a) {
-  static_assert(!(REG && GUM), "Gumbel steps walk their rows in shared memory");
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kPerVec = BF16 ? 8 : 4;
   const StepConfig& cfg = a.cfg;
@@ -1274,8 +1310,8 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
 
   // 3b. Threshold seeding from the first row of every warp that belongs to
   //     the first request, when those rows have more than n children in all
-  //     (read from the shared table).
-  if (shared_rows && !GUM) {  // (Gumbel keys are not bounded by these counts)
+  //     (read from the shared table). Gumbel steps count perturbed scores.
+  if (shared_rows) {
     const int64_t end_first = static_cast<int64_t>(r_first + 1) * a.B_in;  // rows of r_first
     const int nfirst = cq.count < W ? cq.count : W;
     uint32_t nch = 0u;
@@ -1288,9 +1324,20 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
       if (warp < cq.count && meta[warp].x != 0xFF800000u && cq.row(warp) < end_first &&
           bounded_wait(&g.full[0], 0u, &ctl->abort_flag, a.status, kStatusTimeout)) {
         const uint4 m = meta[warp];  // the warp's first row: CTA entry `warp`, stage 0
+        int r0 = 0;
+        uint32_t b0 = 0u;
+        if constexpr (GUM) {  // the draws' counter
+          const int64_t row0 = cq.row(warp);
+          r0 = static_cast<int>(row0 / a.B_in);
+          b0 = static_cast<uint32_t>(row0 - static_cast<int64_t>(r0) * a.B_in);
+        }
         float rmax0, lse0;
         row_stats<BF16>(g.stages, a.V, lane, rmax0, lse0);
-        seed_count<BF16>(a, g.stages, __uint_as_float(m.x), lse0, m.z, m.w, C, whist, lane);
+        if constexpr (GUM)
+          seed_count_gumbel<BF16>(a, g.stages, __uint_as_float(m.x), lse0, m.z, m.w, C, whist,
+                                  lane, r0, b0);
+        else
+          seed_count<BF16>(a, g.stages, __uint_as_float(m.x), lse0, m.z, m.w, C, whist, lane);
       }
       team_sync(team);
       if (warp == 0) {
@@ -1414,11 +1461,21 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         row_stats_reg<BF16, true>(x, nvec, lane, rmax, c.lse);
       else
         row_stats_reg<BF16>(x, nvec, lane, rmax, c.lse);
+      if (GUM && lane == 0) a.row_lse[row] = c.lse;  // the writer recomputes scores from it
       row_thresholds(wb, ctl, req_now);
       float zthr = zthreshold(wb.thr, c.s, c.lse);
-      if (rmax < zthr) continue;
+      if constexpr (GUM) {  // perturbed logits reach at most z + T * kGumbelMax
+        if (rmax + a.gumbel_T * kGumbelMax < zthr) continue;
+      } else {
+        if (rmax < zthr) continue;
+      }
       if (csr) {
-        const bool ok = cin && cz >= zthr;
+        bool ok = cin && cz >= zthr;
+        if constexpr (GUM) {
+          ok = cin && cz + a.gumbel_T * kGumbelMax >= zthr;
+          if (ok) cz += gumbel_noise(a, r, b, ccode);
+          ok = ok && cz >= zthr;
+        }
         if (!__any_sync(kFull, ok)) continue;
         const float score = c.s + (cz - c.lse);
         warp_bin(ctl->hist, ok, score_bin(score, C), wb.binned, &ctl->hist_total);
@@ -1429,15 +1486,16 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
         uint32_t hp[kRegVecs / 4];
         const bool any =
             (full && nparts == 1)
-                ? reg_hits<BF16, true>(a, x, nvec, zthr, hmask, lane, part, nparts, hp)
-                : reg_hits<BF16, false>(a, x, nvec, zthr, hmask, lane, part, nparts, hp);
+                ? reg_hits<BF16, true, GUM>(a, x, nvec, zthr, hmask, lane, part, nparts, hp, r, b)
+                : reg_hits<BF16, false, GUM>(a, x, nvec, zthr, hmask, lane, part, nparts, hp, r,
+                                             b);
         if (!any) continue;
         const int nhits = static_cast<int>(
             __reduce_add_sync(kFull, __popc(hp[0]) + __popc(hp[1]) + __popc(hp[2]) + __popc(hp[3])));
         const uint8_t* zg = a.logits + row * a.row_bytes;
         auto take = [&](int mode) {
-          const TakeOut o = take_hits<BF16>(a, zg, hp[0], hp[1], hp[2], hp[3], hmask, my_prefix, c,
-                                            zthr, wb, ctl, sinks, lane, mode);
+          const TakeOut o = take_hits<BF16, GUM>(a, zg, hp[0], hp[1], hp[2], hp[3], hmask,
+                                                 my_prefix, c, zthr, wb, ctl, sinks, lane, mode);
           wb.thr = o.thr;
           wb.count = o.count;
           wb.binned = o.binned;
@@ -1506,7 +1564,7 @@ static_assert(dev::kHistBins == kPlanHistBins, "the plan sizes the rank-merge sc
 // follows a first eager call).
 static cudaError_t opt_in_smem(const void* fn, int which) {
   static std::mutex mu;
-  static bool done[6][64] = {};
+  static bool done[8][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1580,8 +1638,7 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
   // children (turned into a bitmap).
   const int prefix_words = dense ? a.mask_stride
                                  : (a.layout == SIDBEAM_LAYOUT_CSR ? ((V + 31) / 32 + 3) / 4 * 4 : 0);
-  // (Gumbel steps walk every row in shared memory.)
-  const bool reg = !gum && static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
+  const bool reg = static_cast<int64_t>(V) * esize <= 16 * 32 * kRegVecs;
   const int ctl_bytes = round_up(static_cast<int>(sizeof(dev::SelCtl)), 128);
   if (!choose_step_config(V, esize, extra, prefix_words, n_out, reg, ctl_bytes, &a.cfg) &&
       !(reg && choose_step_config(V, esize, extra, prefix_words, n_out, false, ctl_bytes,
@@ -1592,13 +1649,15 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_step: internal warp plan out of range");
   a.coop = a.part.rows_per_cta < a.cfg.W ? 1 : 0;
 
-  const void* fns[6] = {reinterpret_cast<const void*>(&beam_step_kernel<0, 0>),
+  const void* fns[8] = {reinterpret_cast<const void*>(&beam_step_kernel<0, 0>),
                         reinterpret_cast<const void*>(&beam_step_kernel<1, 0>),
                         reinterpret_cast<const void*>(&beam_step_kernel<0, 1>),
                         reinterpret_cast<const void*>(&beam_step_kernel<1, 1>),
                         reinterpret_cast<const void*>(&beam_step_kernel<0, 0, 1>),
-                        reinterpret_cast<const void*>(&beam_step_kernel<1, 0, 1>)};
-  const int which = (gum ? 4 : (a.cfg.reg ? 2 : 0)) + (a.bf16 ? 1 : 0);
+                        reinterpret_cast<const void*>(&beam_step_kernel<1, 0, 1>),
+                        reinterpret_cast<const void*>(&beam_step_kernel<0, 1, 1>),
+                        reinterpret_cast<const void*>(&beam_step_kernel<1, 1, 1>)};
+  const int which = (gum ? 4 : 0) + (a.cfg.reg ? 2 : 0) + (a.bf16 ? 1 : 0);
   cudaError_t e = opt_in_smem(fns[which], which);
   if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaFuncSetAttribute");
   const dim3 grid(static_cast<unsigned>(a.part.grid));
@@ -1613,7 +1672,9 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
     case 2: beam_step_kernel<0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 3: beam_step_kernel<1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
     case 4: beam_step_kernel<0, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    default: beam_step_kernel<1, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    case 5: beam_step_kernel<1, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    case 6: beam_step_kernel<0, 1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    default: beam_step_kernel<1, 1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "beam_step: launch");
