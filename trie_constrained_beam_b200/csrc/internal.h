@@ -35,7 +35,7 @@ struct sidbeam_trie {
   sidbeam::StepTrie steps[SIDBEAM_MAX_DEPTH];
   int64_t n_leaves = 0;
   int32_t* leaf_rows = nullptr;    // [n_leaves]
-  uint16_t* leaf_codes = nullptr;  // [depth][n_leaves + 8], SoA
+  uint16_t* leaf_codes = nullptr;  // [depth][leaf_codes_stride], SoA (stride: n_leaves rounded up to 8, plus 8)
   int64_t leaf_codes_stride = 0;   // n_leaves + 8
   size_t leaf_bytes = 0;
 };
