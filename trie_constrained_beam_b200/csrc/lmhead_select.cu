@@ -278,6 +278,11 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
     }
     sum = warp_sum(sum);
     const float lse = m + logf(sum);
+    {  // no child of the row can reach the bounds already known: nothing to walk
+      const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&ctl->cta_thr);
+      if (c > wb.thr) wb.thr = c;
+      if (m < zthreshold(wb.thr, s, lse)) return;
+    }
     const uint32_t b = static_cast<uint32_t>(row - static_cast<int64_t>(r) * a.B_in);
     const uint32_t idx0 = b * static_cast<uint32_t>(a.V);
     const uint32_t o0 = a.layout ? a.off[pn] : 0u;
@@ -320,10 +325,19 @@ __global__ void __launch_bounds__(kSelWarps * 32, 1) lmhead_select_kernel(const 
       before = pre + incl - mine;
     }
     // Walk the lane's set bits kBatch at a time (independent logit loads in
-    // flight together; a node may have thousands of children).
-    int cw = l0;
-    uint32_t bits = cw < l1 ? word(cw) : 0u;
+    // flight together; a node may have thousands of children). A lane whose
+    // tiles' largest logits (the GEMM's per-tile maxima) cannot reach the
+    // threshold loads none of its children's logits.
     float zthr = zthreshold(wb.thr, s, lse);
+    int cw = l0;
+    if (l0 < l1) {
+      constexpr int kTileWords = kLmheadTileN / 32;
+      float tmax = __int_as_float(0xFF800000);
+      for (int t = l0 / kTileWords; t <= (l1 - 1) / kTileWords; ++t)
+        tmax = fmaxf(tmax, a.partial[row * a.ntiles + t].x);
+      if (tmax < zthr) cw = l1;
+    }
+    uint32_t bits = cw < l1 ? word(cw) : 0u;
     while (true) {
       int code[kBatch];
       int32_t node[kBatch];
