@@ -1203,6 +1203,11 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
   g.S = S;
   const uint64_t pol = policy_evict_first();
 
+  // 0. Programmatic dependent launch: the next launch on the stream may start
+  //    its own set-up now; this grid touches no global memory before the grid
+  //    it depends on (the previous step, which wrote the parents and cleared
+  //    the workspace counters) has completed and its writes are visible.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // 1. This warp's barriers, and the logits of its first S rows, before any
   //    parent data is known (the rest of each stage follows below).
   if (lane == 0) {
@@ -1210,6 +1215,7 @@ __global__ void __launch_bounds__(REG ? kMaxStepWarpsReg * 32 : kMaxStepWarps * 
     fence_mbar_init();
   }
   __syncwarp();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int spec = q.count < S ? q.count : S;
   if (lane == 0) {
     for (int k = 0; k < spec; ++k) {
@@ -1666,17 +1672,29 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
     e = cudaMemsetAsync(workspace, 0, clear_bytes, stream);
     if (e != cudaSuccess) return cuda_error(e, "beam_step: cudaMemsetAsync");
   }
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (its launch and set-up overlap that kernel's tail; see the kernel's step 0).
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = static_cast<size_t>(a.cfg.smem_bytes);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
   switch (which) {
-    case 0: beam_step_kernel<0, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 1: beam_step_kernel<1, 0><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 2: beam_step_kernel<0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 3: beam_step_kernel<1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 4: beam_step_kernel<0, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 5: beam_step_kernel<1, 0, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    case 6: beam_step_kernel<0, 1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
-    default: beam_step_kernel<1, 1, 1><<<grid, block, a.cfg.smem_bytes, stream>>>(a); break;
+    case 0: e = cudaLaunchKernelEx(&lc, beam_step_kernel<0, 0>, a); break;
+    case 1: e = cudaLaunchKernelEx(&lc, beam_step_kernel<1, 0>, a); break;
+    case 2: e = cudaLaunchKernelEx(&lc, beam_step_kernel<0, 1>, a); break;
+    case 3: e = cudaLaunchKernelEx(&lc, beam_step_kernel<1, 1>, a); break;
+    case 4: e = cudaLaunchKernelEx(&lc, beam_step_kernel<0, 0, 1>, a); break;
+    case 5: e = cudaLaunchKernelEx(&lc, beam_step_kernel<1, 0, 1>, a); break;
+    case 6: e = cudaLaunchKernelEx(&lc, beam_step_kernel<0, 1, 1>, a); break;
+    default: e = cudaLaunchKernelEx(&lc, beam_step_kernel<1, 1, 1>, a); break;
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "beam_step: launch");
   return SIDBEAM_OK;
 }
