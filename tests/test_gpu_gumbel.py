@@ -185,3 +185,26 @@ def test_gumbel_wide_beam_step1_shape(tcb):
     g = _run(tcb, gtrie, 1, z, ps, pn, R, B_in, n, V, T, seed, "bf16")
     ref = oracle.beam_step_gumbel(otrie, 1, z, ps, pn, R, B_in, n, V, T, seed)
     _compare(g, ref, R, n, T, otrie, 1, z, ps, pn, B_in, V, seed)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_gumbel_rows_over_8kb_shared_memory_path(tcb, layout):
+    """fp32 rows of V = 4,096 (16 KB: walked in shared memory, not held in
+    registers), parents with up to ~3,000 children and more rows per CTA than
+    warps, so the perturbed-score seeding of the first rows runs; both trie
+    layouts."""
+    V, R, B_in, n = 4096, 2, 300, 64
+    rng = np.random.default_rng(40 + layout)
+    cat = np.array([(a, c) for a in range(24)
+                    for c in rng.choice(V, size=int(rng.integers(200, 3000)), replace=False)])
+    otrie = oracle.OracleTrie(cat, [V, V])
+    gtrie = tcb.sid_trie_build(cat, [V, V], [layout, layout])
+    M = R * B_in
+    z = (3.0 * rng.standard_normal((M, V))).astype(np.float32)
+    ps = np.concatenate([np.sort(rng.uniform(-8, -1, size=B_in))[::-1] for _ in range(R)])
+    ps = ps.astype(np.float32)
+    pn = rng.integers(0, otrie.n_nodes(1), size=M).astype(np.int32)
+    seed = 0xC0FFEE + layout
+    g = _run(tcb, gtrie, 1, z, ps, pn, R, B_in, n, V, 1.0, seed, "f32")
+    ref = oracle.beam_step_gumbel(otrie, 1, z, ps, pn, R, B_in, n, V, 1.0, seed)
+    _compare(g, ref, R, n, 1.0, otrie, 1, z, ps, pn, B_in, V, seed)
