@@ -535,7 +535,9 @@ int launch_fused_lmhead(const sidbeam_trie* trie, int step, const void* hidden,
   s.part = part;
   int npow2 = 1;
   while (npow2 < n_out) npow2 <<= 1;
-  s.Cw = std::max((n_out + 31) / 32 * 32 + 32, (npow2 + kSelWarps - 1) / kSelWarps / 32 * 32 + 32);
+  // Warp buffers: n plus 512 entries of slack, so that parents with thousands
+  // of children above the bound compact their buffers rarely.
+  s.Cw = std::max((n_out + 31) / 32 * 32 + 512, (npow2 + kSelWarps - 1) / kSelWarps / 32 * 32 + 32);
   s.coop = part.rows_per_cta < kSelWarps ? 1 : 0;
   const size_t smem = ((sizeof(SelCtl) + 127) / 128) * 128 + 1024 + 8192 + kHeavyList * 8 + 128 +
                       static_cast<size_t>(kSelWarps) * s.Cw * 12;
