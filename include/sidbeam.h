@@ -72,7 +72,7 @@ typedef enum {
   SIDBEAM_LAYOUT_CSR = 2    /* per node: child offset range + child codes      */
 } sidbeam_layout;
 
-/* Limits of this build. */
+/* Limits of the library. */
 #define SIDBEAM_MAX_DEPTH 16
 #define SIDBEAM_MAX_V 32768      /* codes per level; also V*sizeof(dtype) <= 64 KiB */
 #define SIDBEAM_MAX_BEAM 4096    /* n_out of beam_step, K of catalog_score_topk     */
