@@ -787,7 +787,6 @@ struct FlushArgs {
   uint64_t* direct_keys;  // staging for ranking a whole request held by this CTA
   int32_t* direct_vals;   //   (null when no free area is available)
   int direct_cap;
-  int read_request_bound = 1;  // 0: the CTA's bound already includes the request's
 };
 
 // Warp-aggregated append position: this lane's slot among the `keep` lanes.
@@ -1060,8 +1059,7 @@ __device__ bool segment_flush(const Team& t, WarpBuf& wb, SelCtl* ctl, const Flu
     const uint64_t hb = hist_bound(ctl->hist, static_cast<uint32_t>(f.n), f.C, t.lane);
     if (t.lane == 0) {
       const unsigned long long g =
-          f.read_request_bound ? *reinterpret_cast<volatile unsigned long long*>(f.request_thr + f.r)
-                               : 0ull;
+          *reinterpret_cast<volatile unsigned long long*>(f.request_thr + f.r);
       const unsigned long long c = ctl->cta_thr;
       unsigned long long K = hb;
       if (g > K) K = g;
