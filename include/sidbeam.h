@@ -253,7 +253,11 @@ int beam_step_noalloc(const sidbeam_trie* trie, int step, const void* logits,
  *  last_node          device i32 [R][n] (the last step's out_node = leaf id).
  *  out_sids           device i32 [R][n][depth]; a padded beam gives all -1.
  *  out_leaf           device i32 [R][n]; -1 for padded beams.
- * The scores are the last step's out_scores (unchanged). Errors: INVALID_ARG, CUDA. */
+ *  n                  1..SIDBEAM_MAX_BEAM (the steps' n_out).
+ * A beam whose parent slot at some step falls outside [0, n) is reported as
+ * padded. Launched as a programmatic dependent of the previous kernel on the
+ * stream. The scores are the last step's out_scores (unchanged). Errors:
+ * INVALID_ARG, CUDA. */
 int beam_finalize(int depth, int R, int n, const int32_t* bp_parent, const int32_t* bp_code,
                   const int32_t* last_node, int32_t* out_sids, int32_t* out_leaf, void* stream);
 

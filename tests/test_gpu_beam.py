@@ -461,6 +461,50 @@ def test_error_conventions(tcb):
     assert _host(o[1]).tolist()[0] == 0    # row 0 (node (0,)) still expanded
 
 
+
+def _synthetic_backpointers(rng, depth, R, n):
+    """Back-pointers of a ranked search: at step t the first v_t ranks are live
+    beams whose parents are live ranks of step t-1 (the root at step 0); the
+    remaining ranks are padding (parent and code -1). Some requests end with
+    fewer live beams than n, one with none at the last step."""
+    bpp = np.full((depth, R, n), -1, dtype=np.int32)
+    bpc = np.full((depth, R, n), -1, dtype=np.int32)
+    node = np.full((R, n), -1, dtype=np.int32)
+    for r in range(R):
+        prev = 1
+        for t in range(depth):
+            if t == depth - 1 and r == R - 1 and R > 1:
+                v = 0
+            else:
+                v = int(rng.integers(1, n + 1)) if r % 2 else n
+            bpp[t, r, :v] = rng.integers(0, prev, size=v)
+            bpc[t, r, :v] = rng.integers(0, 32768, size=v)
+            prev = v
+        node[r, :prev] = rng.integers(0, 1 << 30, size=prev)
+    return bpp, bpc, node
+
+
+@pytest.mark.parametrize("depth,R,n", [(1, 3, 7), (2, 2, 33), (3, 5, 1000), (5, 16, 512),
+                                       (9, 2, 4096), (16, 2, 4096)])
+def test_finalize_synthetic_backpointers_match_oracle(tcb, depth, R, n):
+    """beam_finalize alone against the oracle's backtrack, on back-pointer
+    arrays drawn directly: one to sixteen steps, beams up to the library's
+    maximum (the deepest shapes stage the most parent slots on chip), padded
+    ranks and a request with no live beam. Bit-exact SIDs and leaves."""
+    import torch
+    rng = np.random.default_rng(1000 * depth + n)
+    bpp, bpc, node = _synthetic_backpointers(rng, depth, R, n)
+    d = lambda x: torch.from_numpy(x).cuda()
+    out_sids = torch.full((R, n, depth), 7, dtype=torch.int32, device="cuda")
+    out_leaf = torch.full((R, n), 7, dtype=torch.int32, device="cuda")
+    tcb.beam_finalize(depth, R, n, d(bpp), d(bpc), d(node), out_sids, out_leaf)
+    torch.cuda.synchronize()
+    fin = oracle.beam_finalize(bpp, bpc, np.zeros((R, n)), node)
+    np.testing.assert_array_equal(_host(out_sids), fin["sids"])
+    np.testing.assert_array_equal(_host(out_leaf), fin["leaf"])
+    assert (fin["leaf"] < 0).any() and (fin["leaf"] >= 0).any()
+
+
 # ---------------------------------------------------------------- per-request widths
 def _search_roots(tcb, gtrie, roots, n, depth, V, seed, sigma, widths=None, graph=False):
     """A whole search from the given per-request root hashes (device generator

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include <cstdio>
 #include <cstring>
@@ -44,33 +45,56 @@ int launch_beam_step(const sidbeam_trie* trie, int step, const void* logits, int
 
 namespace {
 
-__global__ void finalize_kernel(int depth, int R, int n, const int32_t* __restrict__ bp_parent,
-                                const int32_t* __restrict__ bp_code,
-                                const int32_t* __restrict__ last_node,
-                                int32_t* __restrict__ out_sids, int32_t* __restrict__ out_leaf) {
-  const int64_t total = static_cast<int64_t>(R) * n;
-  const int64_t plane = total;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / n;
-    int32_t* sid = out_sids + i * depth;
-    const bool live = bp_code[(depth - 1) * plane + i] >= 0;
-    int slot = static_cast<int>(i - r * n);
-    bool ok = live;
-    for (int t = depth - 1; t >= 0; --t) {
-      if (!ok || slot < 0 || slot >= n) {
-        ok = false;
-        sid[t] = -1;
-        continue;
-      }
-      const int64_t at = t * plane + r * n + slot;
-      sid[t] = bp_code[at];
-      slot = bp_parent[at];
-      if (t > 0 && slot < 0) ok = false;
+// One CTA per request. The parent slots of the inner levels 1 .. depth-2 go
+// to shared memory as 16-bit slots (kNoSlot: outside [0, n)), so that each
+// beam's chain of parent lookups runs there; the codes of all levels are then
+// read from global memory together (one independent gather per level).
+constexpr int kFinalizeThreads = 512;
+constexpr uint16_t kNoSlot = 0xFFFFu;
+
+__global__ void __launch_bounds__(kFinalizeThreads)
+    finalize_kernel(int depth, int n, int64_t plane, const int32_t* __restrict__ bp_parent,
+                    const int32_t* __restrict__ bp_code, const int32_t* __restrict__ last_node,
+                    int32_t* __restrict__ out_sids, int32_t* __restrict__ out_leaf) {
+  extern __shared__ uint16_t inner_slot[];  // [depth - 2][n]
+  // Launched as a programmatic dependent of the last step: nothing is read
+  // before that grid has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * n;
+  for (int t = 1; t < depth - 1; ++t)
+    for (int k = threadIdx.x; k < n; k += blockDim.x) {
+      const int32_t p = bp_parent[t * plane + base + k];
+      inner_slot[(t - 1) * n + k] = (p >= 0 && p < n) ? static_cast<uint16_t>(p) : kNoSlot;
     }
-    if (!ok)
-      for (int t = 0; t < depth; ++t) sid[t] = -1;
-    out_leaf[i] = ok ? last_node[i] : -1;
+  __syncthreads();
+  constexpr int kD = SIDBEAM_MAX_DEPTH;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const int64_t i = base + k;
+    const int64_t top = (depth - 1) * plane + i;
+    const int32_t code_top = bp_code[top];
+    const int32_t leaf = last_node[i];
+    int s = depth > 1 ? bp_parent[top] : 0;
+    bool ok = code_top >= 0;  // a padded beam has no code at the last step
+    // Slots of levels depth-2 .. 0, each in [0, n) for a valid beam.
+    int slot[kD - 1];
+#pragma unroll
+    for (int t = kD - 2; t >= 0; --t) {
+      slot[t] = 0;
+      if (t < depth - 1) {
+        if (s < 0 || s >= n) ok = false;
+        if (ok) slot[t] = s;
+        if (t >= 1) s = ok ? static_cast<int>(inner_slot[(t - 1) * n + s]) : -1;
+      }
+    }
+    int32_t code[kD - 1];
+#pragma unroll
+    for (int t = 0; t < kD - 1; ++t)
+      code[t] = (t < depth - 1 && ok) ? bp_code[t * plane + base + slot[t]] : -1;
+    int32_t* sid = out_sids + i * depth;
+#pragma unroll
+    for (int t = 0; t < kD; ++t)
+      if (t < depth) sid[t] = !ok ? -1 : (t == depth - 1 ? code_top : code[t]);
+    out_leaf[i] = ok ? leaf : -1;
   }
 }
 
@@ -222,20 +246,53 @@ extern "C" int beam_step_gumbel(const sidbeam_trie* trie, int step, const void* 
                           seed, row_lse, nullptr, 0);
 }
 
+// Opt the finalize kernel into its largest shared-memory use once per device.
+static cudaError_t finalize_opt_in() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  constexpr int kMax = (SIDBEAM_MAX_DEPTH - 2) * SIDBEAM_MAX_BEAM * 2;
+  if (dev < 0 || dev >= 64)
+    return cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMax);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMax);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
 extern "C" int beam_finalize(int depth, int R, int n, const int32_t* bp_parent,
                              const int32_t* bp_code, const int32_t* last_node, int32_t* out_sids,
                              int32_t* out_leaf, void* stream) {
   if (!bp_parent || !bp_code || !last_node || !out_sids || !out_leaf)
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_finalize: NULL pointer argument");
-  if (depth < 1 || depth > SIDBEAM_MAX_DEPTH || R < 1 || n < 1)
+  if (depth < 1 || depth > SIDBEAM_MAX_DEPTH || R < 1 || n < 1 || n > SIDBEAM_MAX_BEAM)
     return set_error(SIDBEAM_ERR_INVALID_ARG, "beam_finalize: bad shape depth=%d R=%d n=%d",
                      depth, R, n);
-  const int64_t total = static_cast<int64_t>(R) * n;
-  int64_t g = (total + 255) / 256;
-  if (g > 148 * 8) g = 148 * 8;
-  finalize_kernel<<<static_cast<unsigned>(g), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      depth, R, n, bp_parent, bp_code, last_node, out_sids, out_leaf);
-  const cudaError_t e = cudaGetLastError();
+  const size_t smem = static_cast<size_t>(depth > 2 ? depth - 2 : 0) * n * sizeof(uint16_t);
+  cudaError_t e = cudaSuccess;
+  if (smem > 48 * 1024) {
+    e = finalize_opt_in();
+    if (e != cudaSuccess) return cuda_error(e, "beam_finalize: cudaFuncSetAttribute");
+  }
+  const int threads = std::min(kFinalizeThreads, (n + 31) / 32 * 32);
+  // A programmatic dependent of the previous kernel on the stream (the last
+  // beam_step): its launch overlaps that kernel's tail.
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = dim3(static_cast<unsigned>(R));
+  lc.blockDim = dim3(static_cast<unsigned>(threads));
+  lc.dynamicSmemBytes = smem;
+  lc.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, finalize_kernel, depth, n, static_cast<int64_t>(R) * n, bp_parent,
+                         bp_code, last_node, out_sids, out_leaf);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? SIDBEAM_OK : cuda_error(e, "beam_finalize: launch");
 }
 
