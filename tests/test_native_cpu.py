@@ -114,6 +114,26 @@ def test_step_options_argument_checks(lib):
                                       P(0x4000), P(0x5000), P(0x6000), 1 << 20, None) == -1
 
 
+def test_finalize_argument_checks(lib):
+    """beam_finalize rejects bad shapes and NULL pointers on the host, before any
+    device call: depth outside 1..SIDBEAM_MAX_DEPTH, R < 1, n outside
+    1..SIDBEAM_MAX_BEAM (the kernel keeps parent slots in 16 bits)."""
+    P = ctypes.c_void_p
+    ptrs = [P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000)]
+
+    def fin(depth, R, n, p=ptrs):
+        return lib.beam_finalize(depth, R, n, *p, None)
+    assert fin(0, 1, 4) == -1
+    assert fin(17, 1, 4) == -1
+    assert fin(3, 0, 4) == -1
+    assert fin(3, 1, 0) == -1
+    assert fin(3, 1, 4097) == -1
+    for k in range(5):
+        assert fin(3, 1, 4, ptrs[:k] + [None] + ptrs[k + 1:]) == -1
+    from trie_constrained_beam_b200 import native
+    assert "beam_finalize" in native.sidbeam_last_error()
+
+
 def test_header_is_plain_c(tmp_path):
     """include/sidbeam.h compiles on its own as C99 (pedantic): no C++ or CUDA
     types leak into the boundary."""
